@@ -1,0 +1,226 @@
+/*
+ * attn.h -- C ABI of libattn.so: FlashAttention forward and backward for
+ * NVIDIA B200 (sm_100a) with the Generalized Sliding Window mask.
+ *
+ * What the calls compute.  For every sequence b and head h, with
+ * c = sm_scale and the window of the sequence (below):
+ *     S_ij = c * <q_i, k_j>,  LSE_i = ln sum_{allowed j} exp(S_ij),
+ *     P_ij = exp(S_ij - LSE_i) on allowed j (0 elsewhere),  O_i = sum_j P_ij v_j.
+ * A row with no allowed key gets O_i = 0 and LSE_i = -inf.  attn_bwd returns
+ * the gradient of <dO, O> with respect to Q, K and V:
+ *     dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),  dQ = c dS K,  dK = c dS^T Q.
+ * The aotriton README (section "Kernel Support") names this kernel family:
+ * FlashAttention after Tri Dao, which reaches the plain definition above.
+ *
+ * The window (AOTriton 0.10b release notes, "Major Changes from Release 0.9
+ * Beta": causal masks are sliding windows and both window sides may be
+ * negative; AOTriton 0.15b release notes, "Bottom-Right Aligned Sliding
+ * Windows"): with d = seqlen_k - seqlen_q of the sequence,
+ *   - window_left == ATTN_CAUSAL_TOP_LEFT:     key j allowed iff j <= i
+ *   - window_left == ATTN_CAUSAL_BOTTOM_RIGHT: key j allowed iff j <= i + d
+ *     (window_right is ignored for both sentinels, and the diagonal bit
+ *     never shifts a sentinel)
+ *   - otherwise (L, R) = (window_left, window_right) under the TOP_LEFT
+ *     diagonal and (window_left - d, window_right + d) under BOTTOM_RIGHT;
+ *     ATTN_WINDOW_INF on a side leaves it unbounded (and is not shifted);
+ *     key j allowed iff i - L <= j <= i + R (both ends inclusive).
+ * Negative windows are legal; an empty window masks its rows fully.
+ *
+ * Conventions of every call (AOTriton 0.14b release notes, "Runtime Bug
+ * Fixes": the device is taken from the stream, calls do not rely on a
+ * caller-held lock and keep no per-thread caches):
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream of the calling thread's current device).  The device is
+ *     the stream's device, whatever the calling thread's current device is.
+ *   - The caller owns every buffer, the backward workspace included; the
+ *     library allocates no device memory and holds no per-call state, so
+ *     calls from several host threads are safe.
+ *   - Return value: a cudaError_t code.  0 = success.
+ *     ATTN_ERROR_INVALID_VALUE (cudaErrorInvalidValue) for: a wrong
+ *     struct_size / version, reserved VarlenBits set, an unsupported mode,
+ *     dtype or head dimension, a NULL required pointer, a base address not
+ *     16-byte aligned, a stride whose byte size is not a multiple of 16, or a
+ *     backward workspace that is too small.  ATTN_ERROR_NO_KERNEL_IMAGE
+ *     (cudaErrorNoKernelImageForDevice) on a GPU other than sm_100.  Launch
+ *     errors are passed through.  A failing call writes nothing.
+ *   - Tensors: fp16 or bf16 (ATTN_DTYPE_*), the head dimension D contiguous
+ *     (stride 1), D a multiple of 16 in [16, 128].  Strides are in ELEMENTS.
+ *       dense  (BHSD):  element (b, h, s, d) at base + b*stride[0] + h*stride[1]
+ *                       + s*stride[2] + d
+ *       packed (1THD):  element (t, h, d) at base + t*stride[2] + h*stride[1] + d
+ *                       (stride[0] is ignored); token t of sequence b is row
+ *                       cu_seqlens[b] + t.
+ *   - LSE is fp32 in the layout chosen by the VarlenBits lse_layout field:
+ *       HT dense [B, H, Sq], HT packed [H, total_q],
+ *       TH dense [B, Sq, H], TH packed [total_q, H]   (all contiguous).
+ *   - A device-side wait that runs past its iteration limit does not hang or
+ *     trap: the kernel records it in a status word and returns early (the
+ *     output is then invalid).  attn_device_status() reads and clears it.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols keep default visibility even when the library is built
+ * with -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#define ATTN_PARAMS_VERSION 1u
+
+/* Return codes (numeric values of cudaError_t). */
+#define ATTN_SUCCESS 0
+#define ATTN_ERROR_INVALID_VALUE 1
+#define ATTN_ERROR_NO_KERNEL_IMAGE 209
+
+/* Element types of Q, K, V, O, dO, dQ, dK, dV. */
+#define ATTN_DTYPE_FP16 0
+#define ATTN_DTYPE_BF16 1
+
+/* Window encodings (values chosen by this library; the pages name the
+ * sentinel idea, not the numbers). */
+#define ATTN_WINDOW_INF 2147483647
+#define ATTN_CAUSAL_TOP_LEFT (-2147483647 - 1)
+#define ATTN_CAUSAL_BOTTOM_RIGHT (-2147483647)
+
+/*
+ * VarlenBits, one uint32_t (AOTriton 0.14b release notes, "VarlenBits
+ * supersedes VarlenType"; bit 18 from the 0.15b notes, "API Changes"):
+ *   bits  7:0  Q-side VarlenMode    bits 15:8  K-side VarlenMode
+ *   bits 17:16 lse_layout (0 = HT, 1 = TH; 2 and 3 are rejected)
+ *   bit  18    principal diagonal (0 = TOP_LEFT, 1 = BOTTOM_RIGHT)
+ *   bits 31:19 reserved, must be 0.
+ * VarlenMode (one byte): bit 0 stacked (0 = BHSD, 1 = 1THD), bits 2:1 length
+ * (0 uniform, 1 cumulative sums, 2 per-sequence array), bits 4:3 position
+ * (0 uniform, 1 reuse the cumulative sums, 2 second array), bits 7:5
+ * reserved.  Supported: both sides ATTN_VARLEN_MODE_DENSE, or both sides
+ * ATTN_VARLEN_MODE_PACKED; any other mode returns ATTN_ERROR_INVALID_VALUE.
+ */
+#define ATTN_VARLEN_MODE(stacked, length, position) \
+  ((uint32_t)(stacked) | ((uint32_t)(length) << 1) | ((uint32_t)(position) << 3))
+#define ATTN_VARLEN_MODE_DENSE ATTN_VARLEN_MODE(0, 0, 0)
+#define ATTN_VARLEN_MODE_PACKED ATTN_VARLEN_MODE(1, 1, 1)
+#define ATTN_LSE_HT 0u
+#define ATTN_LSE_TH 1u
+#define ATTN_DIAGONAL_TOP_LEFT 0u
+#define ATTN_DIAGONAL_BOTTOM_RIGHT 1u
+#define ATTN_VARLEN_BITS(qmode, kmode, lse_layout, diagonal)                      \
+  ((uint32_t)(qmode) | ((uint32_t)(kmode) << 8) | ((uint32_t)(lse_layout) << 16) | \
+   ((uint32_t)(diagonal) << 18))
+
+/*
+ * Forward parameters.  Sizes: dense -- B batches of Sq queries and Sk keys;
+ * packed -- B sequences, Sq / Sk the largest seqlen_q / seqlen_k (they size
+ * the launch; a sequence longer than them is an error of the caller),
+ * total_q / total_k the rows of the packed tensors, cu_seqlens_q / _k device
+ * arrays of B + 1 int32 cumulative lengths starting at 0.
+ */
+typedef struct attn_fwd_params {
+  uint32_t struct_size; /* sizeof(attn_fwd_params) */
+  uint32_t version;     /* ATTN_PARAMS_VERSION */
+  int32_t dtype;        /* ATTN_DTYPE_FP16 or ATTN_DTYPE_BF16 */
+  int32_t B, H, Sq, Sk, D;
+  int64_t total_q, total_k; /* packed only */
+  const void* q;            /* [B,H,Sq,D] or [total_q,H,D] */
+  const void* k;            /* [B,H,Sk,D] or [total_k,H,D] */
+  const void* v;            /* like k */
+  void* o;                  /* like q, written */
+  float* lse;               /* written; may be NULL (then not written) */
+  int64_t q_stride[3], k_stride[3], v_stride[3], o_stride[3]; /* batch, head, seq */
+  float sm_scale;           /* any finite value, zero and negative included */
+  int32_t window_left, window_right;
+  uint32_t varlen_bits;
+  const int32_t* cu_seqlens_q; /* packed only, device memory */
+  const int32_t* cu_seqlens_k;
+} attn_fwd_params;
+
+/*
+ * Backward parameters: the forward's fields plus the forward output O, its
+ * LSE (same layout as written by attn_fwd, required), the incoming gradient
+ * dO (its own strides: it need not share O's), the outputs dQ / dK / dV and
+ * a caller-owned device workspace of attn_bwd_workspace_size() bytes,
+ * 256-byte aligned.  The workspace holds, after the call, the fp32 rowsums
+ * delta = rowsum(dO o O) [H][rows] followed by the fp32 dQ accumulator
+ * [H][rows][D], rows = B*Sq (dense) or total_q (packed).
+ */
+typedef struct attn_bwd_params {
+  uint32_t struct_size; /* sizeof(attn_bwd_params) */
+  uint32_t version;     /* ATTN_PARAMS_VERSION */
+  int32_t dtype;
+  int32_t B, H, Sq, Sk, D;
+  int64_t total_q, total_k;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  int64_t q_stride[3], k_stride[3], v_stride[3], o_stride[3], do_stride[3];
+  int64_t dq_stride[3], dk_stride[3], dv_stride[3];
+  float sm_scale;
+  int32_t window_left, window_right;
+  uint32_t varlen_bits;
+  const int32_t* cu_seqlens_q;
+  const int32_t* cu_seqlens_k;
+  void* workspace;
+  size_t workspace_bytes;
+} attn_bwd_params;
+
+/* Forward: writes O and (unless lse is NULL) LSE.  One kernel launch. */
+ATTN_API int attn_fwd(const attn_fwd_params* params, void* stream);
+
+/* Backward: writes dQ, dK, dV (and the workspace).  Three kernel launches on
+ * `stream`: rowsum(dO o O) with the dQ accumulator cleared, the main
+ * backward, and the dQ conversion. */
+ATTN_API int attn_bwd(const attn_bwd_params* params, void* stream);
+
+/* Bytes of device workspace attn_bwd needs for these sizes (host only; reads
+ * the size fields, no pointer).  0 if the sizes are invalid. */
+ATTN_API size_t attn_bwd_workspace_size(const attn_bwd_params* params);
+
+/* Number of allowed (query, key) pairs of one sequence under a window, the
+ * unit of the FLOP counts (4*D per pair forward, 10*D backward).  Host only. */
+ATTN_API int64_t attn_allowed_pairs(int32_t seqlen_q, int32_t seqlen_k, int32_t window_left,
+                           int32_t window_right, uint32_t bottom_right);
+
+/*
+ * The kernels' tile plan, computed on the host by the same code the kernels
+ * run, for tests and tools.  For the query tile [m0, m0 + 128) of a sequence
+ * (seqlen_q, seqlen_k) it writes the half-open range of 128-key tiles the
+ * forward visits, *n_begin / *n_end, and for each tile n in the range
+ * full_mask[n - n_begin] = 1 if no element of the tile is masked (the kernel
+ * then skips the element test), 0 otherwise; full_mask needs room for
+ * ceil(seqlen_k / 128) bytes.  Returns 0, or ATTN_ERROR_INVALID_VALUE.
+ */
+ATTN_API int attn_tile_plan(int32_t seqlen_q, int32_t seqlen_k, int32_t window_left,
+                   int32_t window_right, uint32_t bottom_right, int32_t m0, int32_t* n_begin,
+                   int32_t* n_end, uint8_t* full_mask);
+
+/* The backward's mirror: for the key tile [n0, n0 + 128), the half-open range
+ * of 128-query tiles that see any of its keys. */
+ATTN_API int attn_tile_plan_bwd(int32_t seqlen_q, int32_t seqlen_k, int32_t window_left,
+                       int32_t window_right, uint32_t bottom_right, int32_t n0,
+                       int32_t* m_begin, int32_t* m_end);
+
+/* Reads and clears the device status word of the stream's device (waits for
+ * the stream).  *status = 0 when every device-side wait finished in time;
+ * otherwise bit k marks wait site k that gave up.  Returns a cudaError_t. */
+ATTN_API int attn_device_status(void* stream, uint32_t* status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -137,18 +137,24 @@ def _probs_block(q, k, sm_scale, mask):
     return p, lse
 
 
-def forward(q, k, v, sm_scale, window_left, window_right, bottom_right=False):
-    """One (sequence, head): q [Sq, D], k [Sk, D], v [Sk, Dv] -> (O, LSE)."""
+def forward(q, k, v, sm_scale, window_left, window_right, bottom_right=False, rows=None):
+    """One (sequence, head): q [Sq, D], k [Sk, D], v [Sk, Dv] -> (O, LSE).
+
+    ``rows`` (optional) computes only those query rows (each row of the
+    definition depends on its own query only) and returns [len(rows), ...].
+    """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     sq, sk = q.shape[0], k.shape[0]
-    o = np.zeros((sq, v.shape[1]), dtype=np.float64)
-    lse = np.full(sq, -np.inf, dtype=np.float64)
-    for r0 in range(0, sq, ROW_BLOCK):
-        r1 = min(r0 + ROW_BLOCK, sq)
-        mask = allowed(sq, sk, window_left, window_right, bottom_right, np.arange(r0, r1))
-        p, lse[r0:r1] = _probs_block(q[r0:r1], k, sm_scale, mask)
+    idx = np.arange(sq) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = np.zeros((len(idx), v.shape[1]), dtype=np.float64)
+    lse = np.full(len(idx), -np.inf, dtype=np.float64)
+    for r0 in range(0, len(idx), ROW_BLOCK):
+        r1 = min(r0 + ROW_BLOCK, len(idx))
+        sel = idx[r0:r1]
+        mask = allowed(sq, sk, window_left, window_right, bottom_right, sel)
+        p, lse[r0:r1] = _probs_block(q[sel], k, sm_scale, mask)
         o[r0:r1] = p @ v
     return o, lse
 

@@ -1,0 +1,499 @@
+// FlashAttention backward for sm_100a: gradient of <dO, O> for the masked
+// softmax attention the forward computes.
+//
+// Three launches on the caller's stream:
+//  1. attn_bwd_pre_kernel   delta = rowsum(dO o O) in fp32 (the 0.14b release
+//                           notes, "Minor Changes", name this step
+//                           bwd_preprocess, with varlen folded in) and a
+//                           cleared fp32 dQ accumulator;
+//  2. attn_bwd_kernel       one CTA per (128-key tile, head, sequence); it
+//                           keeps K, V and the dK, dV accumulators on chip and
+//                           walks the 128-query tiles whose window reaches its
+//                           keys: S^T = K Q^T, dP^T = V dO^T, P^T and
+//                           dS^T = P^T o (dP^T - delta) in TMEM, dV += P^T dO,
+//                           dK += dS^T Q, dQ_tile = dS K added into the fp32
+//                           accumulator.  dO has strides of its own (the 0.14b
+//                           notes, "Kernel Bug Fixes", record a kernel that
+//                           addressed dO with O's strides);
+//  3. attn_dq_convert_kernel  dQ = sm_scale * accumulator in the input dtype.
+// Warp roles of (2): warps 0-3 "ds" (one key row per thread: P, dS, epilogue),
+// warps 4-7 dQ drain (one query row per thread), warp 8 TMA, warp 9 MMA.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "fwd.h"
+#include "mask.cuh"
+
+namespace attn {
+
+// ---------------------------------------------------------------------------
+// 1. preprocess: 16 threads per (head, row), 8 elements each.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int64_t row_offset(const int64_t* st, int64_t row, int h, int Sq,
+                                              bool packed) {
+  if (packed) return row * st[2] + (int64_t)h * st[1];
+  const int64_t b = row / Sq, s = row % Sq;
+  return b * st[0] + (int64_t)h * st[1] + s * st[2];
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant__ BwdArgs a) {
+  const int64_t n_groups = (int64_t)a.H * a.rows;
+  const int sub = threadIdx.x & 15;
+  const int chunks = a.D / 8;
+  for (int64_t g = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4); g < n_groups;
+       g += (int64_t)gridDim.x * 16) {
+    const int h = (int)(g / a.rows);
+    const int64_t row = g % a.rows;
+    float acc = 0.f;
+    if (sub < chunks) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint8_t*>(a.o) +
+          2 * (row_offset(a.o_stride, row, h, a.Sq, a.packed) + 8 * sub));
+      const uint4 dv = *reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint8_t*>(a.dout) +
+          2 * (row_offset(a.do_stride, row, h, a.Sq, a.packed) + 8 * sub));
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = unpack2<BF16>(ow[e]), y = unpack2<BF16>(dw[e]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(a.dq_acc + g * a.D + 8 * sub);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int m = 8; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (sub == 0) a.delta[g] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. dQ conversion.
+// ---------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_constant__ BwdArgs a) {
+  const int chunks = a.D / 8;
+  const int64_t n = (int64_t)a.H * a.rows * chunks;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n;
+       x += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t g = x / chunks;
+    const int c = (int)(x % chunks);
+    const int h = (int)(g / a.rows);
+    const int64_t row = g % a.rows;
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + g * a.D + 8 * c);
+    const float4 u = src[0], v = src[1];
+    const float s = a.sm_scale;
+    uint8_t* dst = reinterpret_cast<uint8_t*>(a.dq) +
+                   2 * (row_offset(a.dq_stride, row, h, a.Sq, a.packed) + 8 * c);
+    st_global_v4(dst, pack2<BF16>(u.x * s, u.y * s), pack2<BF16>(u.z * s, u.w * s),
+                 pack2<BF16>(v.x * s, v.y * s), pack2<BF16>(v.z * s, v.w * s));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. main backward
+// ---------------------------------------------------------------------------
+template <int DPAD>
+struct BwdCfg {
+  static constexpr int kThreads = 320;
+  static constexpr int kLoadWarp = 8;
+  static constexpr int kMmaWarp = 9;
+  static constexpr int kBlocks = DPAD / 64;
+  static constexpr int kTileBytes = 128 * DPAD * 2;
+  static constexpr int kQStages = 2;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;
+  static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
+  static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;  // 128 x 128 16-bit
+  static constexpr int kOffRow = kOffDS + 128 * 128 * 2;          // lse/delta [2][2][128] f32
+  static constexpr int kOffBar = kOffRow + 2 * 2 * 128 * 4;
+  // kv_full, q_full[QS], q_empty[QS], do_full[QS], do_empty[QS], s_full,
+  // dp_full, p_ready, dq_mma, dq_free, acc_done
+  static constexpr int kNumBars = 1 + 4 * kQStages + 6;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + DPAD;
+  static constexpr bool kAliasDQ = (DPAD == 128);  // dQ tile reuses the dP^T columns
+  static constexpr int kColDQ = kAliasDQ ? kColDP : 256 + 2 * DPAD;
+  static constexpr int kTmemCols = 512;
+};
+
+template <int DPAD, bool BF16>
+__global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
+  using C = BwdCfg<DPAD>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int ntile = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  int32_t sq = a.Sq, sk = a.Sk, qrow0 = 0, krow0 = 0, bcoord = b;
+  if (a.packed) {
+    qrow0 = a.cu_q[b];
+    krow0 = a.cu_k[b];
+    sq = a.cu_q[b + 1] - qrow0;
+    sk = a.cu_k[b + 1] - krow0;
+    bcoord = 0;
+  }
+  const int32_t n0 = ntile * 128;
+  if (n0 >= sk) return;
+  if (sbase & 1023) {  // the swizzled tiles need 1 KiB alignment
+    if (threadIdx.x == 0) atomicOr(a.status, 1u << kSiteTeardown);
+    return;
+  }
+  const SeqWindow win = seq_window(a.wl, a.wr, a.bottom_right != 0, sq, sk);
+  int32_t mb, me;
+  bwd_tile_range(win, sq, sk, n0, &mb, &me);
+  const int n_it = me - mb;
+
+  auto kv_row_ptr = [&](void* base, const int64_t* st, int32_t j) -> uint8_t* {
+    int64_t off = a.packed ? (int64_t)(krow0 + j) * st[2]
+                           : (int64_t)b * st[0] + (int64_t)j * st[2];
+    off += (int64_t)h * st[1];
+    return reinterpret_cast<uint8_t*>(base) + 2 * off;
+  };
+
+  if (n_it <= 0) {
+    // No query sees these keys: dK = dV = 0.
+    const int rows = min(128, sk - n0);
+    for (int idx = threadIdx.x; idx < rows * (a.D / 8); idx += blockDim.x) {
+      const int r = idx / (a.D / 8), c = idx % (a.D / 8);
+      st_global_v4(kv_row_ptr(a.dk, a.dk_stride, n0 + r) + 16 * c, 0u, 0u, 0u, 0u);
+      st_global_v4(kv_row_ptr(a.dv, a.dv_stride, n0 + r) + 16 * c, 0u, 0u, 0u, 0u);
+    }
+    return;
+  }
+
+  const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV, sQ = sbase + C::kOffQ,
+                 sDO = sbase + C::kOffDO, sDS = sbase + C::kOffDS;
+  float* row_s = reinterpret_cast<float*>(smem + C::kOffRow);  // [buf][lse|delta][128]
+  const uint32_t bar0 = sbase + C::kOffBar;
+  const uint32_t kv_full = bar0;
+  auto q_full = [&](int s) { return bar0 + 8 * (1 + s); };
+  auto q_empty = [&](int s) { return bar0 + 8 * (1 + C::kQStages + s); };
+  auto do_full = [&](int s) { return bar0 + 8 * (1 + 2 * C::kQStages + s); };
+  auto do_empty = [&](int s) { return bar0 + 8 * (1 + 3 * C::kQStages + s); };
+  const uint32_t s_full = bar0 + 8 * (1 + 4 * C::kQStages);
+  const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, dq_mma = s_full + 24,
+                 dq_free = s_full + 32, acc_done = s_full + 40;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < C::kQStages; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+      mbar_init(do_full(s), 1);
+      mbar_init(do_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(dq_mma, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::kLoadWarp) {
+    // ===================== TMA producer =====================
+    if (lane == 0) {
+      prefetch_tmap(&a.tq);
+      prefetch_tmap(&a.tk);
+      prefetch_tmap(&a.tv);
+      prefetch_tmap(&a.tdo);
+      mbar_expect_tx(kv_full, 2 * C::kTileBytes);
+      for (int blk = 0; blk < C::kBlocks; ++blk) {
+        tma_load_4d(sK + blk * 16384, &a.tk, kv_full, 64 * blk, krow0 + n0, h, bcoord);
+        tma_load_4d(sV + blk * 16384, &a.tv, kv_full, 64 * blk, krow0 + n0, h, bcoord);
+      }
+      int nq = 0, ndo = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int qs = it % C::kQStages, round = it / C::kQStages;
+        const int qrow = qrow0 + (mb + it) * 128;
+        if (round > 0 && !mbar_wait(q_empty(qs), (round - 1) & 1, abort_flag, a.status, kSiteLoad))
+          break;
+        mbar_expect_tx(q_full(qs), C::kTileBytes);
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sQ + qs * C::kTileBytes + blk * 16384, &a.tq, q_full(qs), 64 * blk, qrow, h,
+                      bcoord);
+        ++nq;
+        if (round > 0 && !mbar_wait(do_empty(qs), (round - 1) & 1, abort_flag, a.status, kSiteLoad))
+          break;
+        mbar_expect_tx(do_full(qs), C::kTileBytes);
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sDO + qs * C::kTileBytes + blk * 16384, &a.tdo, do_full(qs), 64 * blk, qrow,
+                      h, bcoord);
+        ++ndo;
+      }
+      if (*abort_flag) {
+        mbar_wait(kv_full, 0, abort_flag, a.status, kSiteTeardown);
+        for (int it = max(0, nq - C::kQStages); it < nq; ++it)
+          mbar_wait(q_full(it % C::kQStages), (it / C::kQStages) & 1, abort_flag, a.status,
+                    kSiteTeardown);
+        for (int it = max(0, ndo - C::kQStages); it < ndo; ++it)
+          mbar_wait(do_full(it % C::kQStages), (it / C::kQStages) & 1, abort_flag, a.status,
+                    kSiteTeardown);
+      }
+    }
+  } else if (warp == C::kMmaWarp) {
+    // ===================== MMA issuer =====================
+    if (lane == 0) {
+      const uint32_t idesc_kk = make_idesc(BF16, 128, 128, false, false);   // S^T, dP^T
+      const uint32_t idesc_acc = make_idesc(BF16, 128, a.D, false, true);  // dV, dK (A in TMEM)
+      const uint32_t idesc_dq = make_idesc(BF16, 128, a.D, true, true);    // dQ = dS K
+      const int ksteps = a.D / 16;
+      bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int qs = it % C::kQStages;
+        const uint32_t par = (it / C::kQStages) & 1;
+        const uint32_t qb = sQ + qs * C::kTileBytes, dob = sDO + qs * C::kTileBytes;
+        if (!(ok = mbar_wait(q_full(qs), par, abort_flag, a.status, kSiteMma))) break;
+        tc_fence_after();
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + C::kColS, make_sdesc(sK + off, 16, 1024), make_sdesc(qb + off, 16, 1024),
+                 idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        if (!(ok = mbar_wait(do_full(qs), par, abort_flag, a.status, kSiteMma))) break;
+        if (C::kAliasDQ && it > 0 &&
+            !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag, a.status, kSiteMma)))
+          break;
+        tc_fence_after();
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + C::kColDP, make_sdesc(sV + off, 16, 1024), make_sdesc(dob + off, 16, 1024),
+                 idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(dp_full);
+        if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
+        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tmem + C::kColDV, tmem + C::kColS + 8 * kk, make_sdesc(dob + kk * 2048, 16384, 1024),
+                 idesc_acc, acc);
+          mma_ts(tmem + C::kColDK, tmem + C::kColDP + 8 * kk, make_sdesc(qb + kk * 2048, 16384, 1024),
+                 idesc_acc, acc);
+        }
+        tc_commit(q_empty(qs));
+        tc_commit(do_empty(qs));
+        if (!C::kAliasDQ && it > 0 &&
+            !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag, a.status, kSiteMma)))
+          break;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::kColDQ, make_sdesc(sDS + kk * 2048, 16384, 1024),
+                 make_sdesc(sK + kk * 2048, 16384, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+        tc_commit(dq_mma);
+      }
+      tc_commit(acc_done);
+    }
+  } else if (warp < 4) {
+    // ===================== P, dS and the dK / dV epilogue =====================
+    const int r = warp * 32 + lane;  // key row within the tile
+    const int32_t j = n0 + r;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
+    const float sl2 = a.scale_log2;
+    // Queries that see key j: j - R <= i <= j + L, 0 <= i < sq (none if j >= sk).
+    int32_t qa = j - win.R, qz = j + win.L;
+    if (qa < 0) qa = 0;
+    if (qz > sq - 1) qz = sq - 1;
+    if (j >= sk) qz = qa - 1;
+    auto row_vals = [&](int it, float& lse, float& dl) {
+      const int32_t i = (mb + it) * 128 + r;
+      lse = 0.f;
+      dl = 0.f;
+      if (i < sq) {
+        int64_t li;
+        if (a.packed)
+          li = a.lse_th ? (int64_t)(qrow0 + i) * a.H + h : (int64_t)h * a.total_q + qrow0 + i;
+        else
+          li = a.lse_th ? ((int64_t)b * a.Sq + i) * a.H + h : ((int64_t)b * a.H + h) * a.Sq + i;
+        lse = a.lse[li] * 1.4426950408889634f;
+        const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
+        dl = a.delta[(int64_t)h * a.rows + row];
+      }
+    };
+    float lse_n, dl_n;
+    row_vals(0, lse_n, dl_n);
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int buf = it & 1;
+      float* lse_s = row_s + buf * 256;
+      float* dl_s = lse_s + 128;
+      lse_s[r] = lse_n;
+      dl_s[r] = dl_n;
+      // Every warp of the group passes this barrier once per tile, aborted or
+      // not, so none can be left waiting at it.
+      named_bar_sync(1, 128);
+      if (!ok) continue;
+      if (it + 1 < n_it) row_vals(it + 1, lse_n, dl_n);
+      const int32_t m0 = (mb + it) * 128;
+      const bool full = tile_is_full(win, sq, sk, m0, n0);
+      const int32_t ca = qa - m0, cz = qz - m0;  // allowed columns [ca, cz]
+      ok = mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
+           mbar_wait(dp_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
+           (it == 0 || mbar_wait(dq_mma, (it - 1) & 1, abort_flag, a.status, kSiteSoftmax));
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tS + 32 * c, sr);
+        tmem_ld32(tDP + 32 * c, dr);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q0 = 32 * c + 2 * e, q1 = q0 + 1;
+          float p0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lse_s[q0]));
+          float p1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lse_s[q1]));
+          if (!full) {
+            p0 = (q0 < ca || q0 > cz) ? 0.f : p0;
+            p1 = (q1 < ca || q1 > cz) ? 0.f : p1;
+          }
+          const float d0 = p0 * (__uint_as_float(dr[2 * e]) - dl_s[q0]);
+          const float d1 = p1 * (__uint_as_float(dr[2 * e + 1]) - dl_s[q1]);
+          pp[e] = pack2<BF16>(p0, p1);
+          dd[e] = pack2<BF16>(d0, d1);
+        }
+        tmem_st16(tS + 16 * c, pp);
+        tmem_st16(tDP + 16 * c, dd);
+        // dS (query-contiguous rows of this key) into the MN-major smem tile.
+        const uint32_t rowb = sDS + (c >> 1) * 16384 + r * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = ((c & 1) * 4 + u) ^ (r & 7);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + chunk * 16),
+                       "r"(dd[4 * u]), "r"(dd[4 * u + 1]), "r"(dd[4 * u + 2]), "r"(dd[4 * u + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, a.status, kSiteEpilogue));
+    if (ok) {
+      tc_fence_after();
+      const bool valid = j < sk;
+      uint8_t* dvrow = valid ? kv_row_ptr(a.dv, a.dv_stride, j) : nullptr;
+      uint8_t* dkrow = valid ? kv_row_ptr(a.dk, a.dk_stride, j) : nullptr;
+      for (int c = 0; c < a.D / 16; ++c) {
+        uint32_t rv[16], rk[16], pv[8], pk[8];
+        tmem_ld16(tmem + lane_off + C::kColDV + 16 * c, rv);
+        tmem_ld16(tmem + lane_off + C::kColDK + 16 * c, rk);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pv[e] = pack2<BF16>(__uint_as_float(rv[2 * e]), __uint_as_float(rv[2 * e + 1]));
+          pk[e] = pack2<BF16>(__uint_as_float(rk[2 * e]) * a.sm_scale,
+                              __uint_as_float(rk[2 * e + 1]) * a.sm_scale);
+        }
+        if (valid) {
+          st_global_v4(dvrow + 32 * c, pv[0], pv[1], pv[2], pv[3]);
+          st_global_v4(dvrow + 32 * c + 16, pv[4], pv[5], pv[6], pv[7]);
+          st_global_v4(dkrow + 32 * c, pk[0], pk[1], pk[2], pk[3]);
+          st_global_v4(dkrow + 32 * c + 16, pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    }
+  } else {
+    // ===================== dQ drain (warps 4-7) =====================
+    const int quad = warp & 3;
+    const int q = quad * 32 + lane;  // query row within the tile
+    const uint32_t tDQ = tmem + ((uint32_t)(quad * 32) << 16) + C::kColDQ;
+    for (int it = 0; it < n_it; ++it) {
+      bool ok = mbar_wait(dq_mma, it & 1, abort_flag, a.status, kSiteDq);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int32_t i = (mb + it) * 128 + q;
+      const bool valid = i < sq;
+      const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
+      float* dst = a.dq_acc + ((int64_t)h * a.rows + row) * a.D;
+      for (int c = 0; c < a.D / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tDQ + 16 * c, v);
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            red_add_v4(dst + 16 * c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int DPAD, bool BF16>
+static cudaError_t launch_main(const BwdArgs& a, cudaStream_t stream) {
+  using C = BwdCfg<DPAD>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  auto kern = attn_bwd_kernel<DPAD, BF16>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.Sk + 127) / 128, a.H, a.B);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <bool BF16>
+static cudaError_t launch_all(const BwdArgs& a, cudaStream_t stream, int sms) {
+  const int64_t groups = (int64_t)a.H * a.rows;
+  if (groups > 0) {
+    const int64_t want = (groups + 15) / 16;
+    const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+    attn_bwd_pre_kernel<BF16><<<grid, 256, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (a.Sk > 0 && a.H > 0 && a.B > 0) {
+    cudaError_t e = a.D <= 64 ? launch_main<64, BF16>(a, stream) : launch_main<128, BF16>(a, stream);
+    if (e != cudaSuccess) return e;
+  }
+  if (groups > 0) {
+    const int64_t n = groups * (a.D / 8);
+    const int64_t want = (n + 255) / 256;
+    const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+    attn_dq_convert_kernel<BF16><<<grid, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return a.bf16 ? launch_all<true>(a, stream, sms) : launch_all<false>(a, stream, sms);
+}
+
+}  // namespace attn

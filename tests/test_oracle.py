@@ -383,3 +383,12 @@ def test_planted_window_sign_is_caught_by_golden():
         if not np.array_equal(_planted_window_sign(c["sq"], c["sk"], c["wl"], c["wr"], c["br"]), want):
             caught = True
     assert caught
+
+
+def test_row_subset_equals_full_rows():
+    q, k, v = _rand((300, 4), 90), _rand((260, 4), 91), _rand((260, 4), 92)
+    o, lse = ref.forward(q, k, v, 0.4, 50, 3, True)
+    rows = [0, 7, 128, 299]
+    o2, lse2 = ref.forward(q, k, v, 0.4, 50, 3, True, rows=rows)
+    np.testing.assert_array_equal(o2, o[rows])
+    np.testing.assert_array_equal(lse2, lse[rows])
