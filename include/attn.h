@@ -176,6 +176,10 @@ typedef struct attn_bwd_params {
   const int32_t* cu_seqlens_k;
   void* workspace;
   size_t workspace_bytes;
+  /* Optional measurement hook: two cudaEvent_t created by the caller on the
+   * stream's device, recorded on `stream` immediately before and after the
+   * main backward kernel (so the caller can time it alone).  NULL: none. */
+  void* main_kernel_events[2];
 } attn_bwd_params;
 
 /* Forward: writes O and (unless lse is NULL) LSE.  One kernel launch. */

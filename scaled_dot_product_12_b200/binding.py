@@ -73,6 +73,7 @@ class BwdParams(ctypes.Structure):
         ("window_right", ctypes.c_int32), ("varlen_bits", ctypes.c_uint32),
         ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("main_kernel_events", ctypes.c_void_p * 2),
     ]
 
 

@@ -310,6 +310,8 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     a.delta = static_cast<float*>(p->workspace);
     a.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(p->workspace) + delta_bytes);
     a.status = info.status;
+    a.main_events[0] = static_cast<cudaEvent_t>(p->main_kernel_events[0]);
+    a.main_events[1] = static_cast<cudaEvent_t>(p->main_kernel_events[1]);
     return attn::launch_bwd(a, stream);
   });
 }

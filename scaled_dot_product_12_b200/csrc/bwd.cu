@@ -476,8 +476,11 @@ static cudaError_t launch_all(const BwdArgs& a, cudaStream_t stream, int sms) {
     if (e != cudaSuccess) return e;
   }
   if (a.Sk > 0 && a.H > 0 && a.B > 0) {
-    cudaError_t e = a.D <= 64 ? launch_main<64, BF16>(a, stream) : launch_main<128, BF16>(a, stream);
+    cudaError_t e = cudaSuccess;
+    if (a.main_events[0] && (e = cudaEventRecord(a.main_events[0], stream)) != cudaSuccess) return e;
+    e = a.D <= 64 ? launch_main<64, BF16>(a, stream) : launch_main<128, BF16>(a, stream);
     if (e != cudaSuccess) return e;
+    if (a.main_events[1] && (e = cudaEventRecord(a.main_events[1], stream)) != cudaSuccess) return e;
   }
   if (groups > 0) {
     const int64_t n = groups * (a.D / 8);

@@ -43,6 +43,7 @@ struct BwdArgs {
   float* delta;           // workspace: [H][rows]
   float* dq_acc;          // workspace: [H][rows][D]
   uint32_t* status;
+  cudaEvent_t main_events[2];  // optional, recorded around the main kernel
 };
 
 cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream);
