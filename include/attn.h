@@ -194,6 +194,31 @@ ATTN_API int attn_bwd(const attn_bwd_params* params, void* stream);
  * the size fields, no pointer).  0 if the sizes are invalid. */
 ATTN_API size_t attn_bwd_workspace_size(const attn_bwd_params* params);
 
+/*
+ * attn_bwd without a caller-provided workspace (the pages have no counterpart
+ * of this call; it serves callers of this library that cannot allocate device
+ * memory: hosts that own all device memory and hand a kernel library no
+ * allocator, and latency-critical paths where cudaMalloc's implicit
+ * synchronisation is not acceptable).
+ *
+ * The backward's scratch memory (fp32 row sums and the fp32 dQ accumulator)
+ * comes from a device array compiled into the library, ATTN_STATIC_WORKSPACE_BYTES
+ * bytes, which every GPU that loads the library holds until the process exits.
+ * The caller passes inputs and outputs only; params->workspace and
+ * params->workspace_bytes are ignored.  The call allocates nothing.
+ *   - Sizes whose attn_bwd_workspace_size() exceeds ATTN_STATIC_WORKSPACE_BYTES
+ *     are rejected with cudaErrorMemoryAllocation (2) before any GPU work;
+ *     otherwise the return codes are those of attn_bwd.
+ *   - The first call on a device looks up that device's address of the array
+ *     (once per device); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     there; each call clears the accumulator it needs before use.  Calls whose
+ *     work overlaps on the GPU (different streams without ordering between
+ *     them) race on the array and give wrong results: order them.
+ */
+#define ATTN_STATIC_WORKSPACE_BYTES (64u << 20)
+ATTN_API int attn_bwd_static_workspace(const attn_bwd_params* params, void* stream);
+
 /* Number of allowed (query, key) pairs of one sequence under a window, the
  * unit of the FLOP counts (4*D per pair forward, 10*D backward).  Host only. */
 ATTN_API int64_t attn_allowed_pairs(int32_t seqlen_q, int32_t seqlen_k, int32_t window_left,

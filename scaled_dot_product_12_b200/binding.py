@@ -28,6 +28,8 @@ LSE_HT, LSE_TH = 0, 1
 DIAGONAL_TOP_LEFT, DIAGONAL_BOTTOM_RIGHT = 0, 1
 ERROR_INVALID_VALUE = 1
 ERROR_NO_KERNEL_IMAGE = 209
+ERROR_MEMORY_ALLOCATION = 2
+STATIC_WORKSPACE_BYTES = 64 << 20
 
 
 def varlen_mode(stacked: int, length: int, position: int) -> int:
@@ -81,6 +83,7 @@ EXPORTS = {
     "attn_fwd": (ctypes.c_int, [ctypes.POINTER(FwdParams), ctypes.c_void_p]),
     "attn_bwd": (ctypes.c_int, [ctypes.POINTER(BwdParams), ctypes.c_void_p]),
     "attn_bwd_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(BwdParams)]),
+    "attn_bwd_static_workspace": (ctypes.c_int, [ctypes.POINTER(BwdParams), ctypes.c_void_p]),
     "attn_allowed_pairs": (ctypes.c_int64, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                             ctypes.c_int32, ctypes.c_uint32]),
     "attn_tile_plan": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
