@@ -112,15 +112,46 @@ struct BwdCfg {
   static constexpr int kOffRow = kOffDS + 128 * 128 * 2;          // lse/delta [2][2][128] f32
   static constexpr int kOffBar = kOffRow + 2 * 2 * 128 * 4;
   // kv_full, q_full[QS], q_empty[QS], do_full[QS], do_empty[QS], s_full,
-  // dp_full, p_ready, dq_mma, dq_free, acc_done
-  static constexpr int kNumBars = 1 + 4 * kQStages + 6;
+  // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done
+  static constexpr int kNumBars = 1 + 4 * kQStages + 7;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + DPAD;
   static constexpr bool kAliasDQ = (DPAD == 128);  // dQ tile reuses the dP^T columns
   static constexpr int kColDQ = kAliasDQ ? kColDP : 256 + 2 * DPAD;
+  static constexpr bool kDqTransposed = (DPAD == 128);  // dQ^T = K^T dS^T, lane = head dim
   static constexpr int kTmemCols = 512;
 };
+
+// D = A B^T with both operands K-major (A: 128 rows, B: 128 rows, K = head
+// dim): 16-column K steps are +32 bytes inside a 64-column block, blocks
+// 16 KiB apart; padded head-dim columns are zero in both operands.
+template <int KSTEPS>
+__device__ __forceinline__ void bwd_issue_kmajor(uint32_t d, uint32_t a_lo, uint32_t b_lo,
+                                                 uint32_t hi, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk) {
+    const uint32_t o = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+    mma_ss2(d, a_lo + o, hi, b_lo + o, hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+// D (+)= A(TMEM, 128 lanes x 128 K as 16-bit pairs) B(MN-major smem), K = 128.
+__device__ __forceinline__ void bwd_issue_ts(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t hi,
+                                             uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts2(d, a + 8 * kk, b_lo + (uint32_t)(kk * 2048 >> 4), hi, idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
+// D = A B with both operands MN-major in smem, K = 128 (16 rows = 2048 bytes).
+__device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                             uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t o = (uint32_t)(kk * 2048 >> 4);
+    mma_ss2(d, a_lo + o, hi, b_lo + o, hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
 
 template <int DPAD, bool BF16>
 __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
@@ -180,8 +211,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
   auto do_full = [&](int s) { return bar0 + 8 * (1 + 2 * C::kQStages + s); };
   auto do_empty = [&](int s) { return bar0 + 8 * (1 + 3 * C::kQStages + s); };
   const uint32_t s_full = bar0 + 8 * (1 + 4 * C::kQStages);
-  const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, dq_mma = s_full + 24,
-                 dq_free = s_full + 32, acc_done = s_full + 40;
+  const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24,
+                 dq_mma = s_full + 32, dq_free = s_full + 40, acc_done = s_full + 48;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -196,6 +227,7 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_ready, 128);
+    mbar_init(ds_ready, 128);
     mbar_init(dq_mma, 1);
     mbar_init(dq_free, 128);
     mbar_init(acc_done, 1);
@@ -254,53 +286,78 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
     }
   } else if (warp == C::kMmaWarp) {
     // ===================== MMA issuer =====================
+    // Order per query tile `it`:  dV(it), S(it+1), dK(it), dQ(it), dP(it+1).
+    // S(it+1) reuses the S/P columns as soon as dV(it) has read P(it); the
+    // P / dS warps work on tile it+1's P while dK(it) and dQ(it) run.
     if (lane == 0) {
       const uint32_t idesc_kk = make_idesc(BF16, 128, 128, false, false);   // S^T, dP^T
       const uint32_t idesc_acc = make_idesc(BF16, 128, a.D, false, true);  // dV, dK (A in TMEM)
-      const uint32_t idesc_dq = make_idesc(BF16, 128, a.D, true, true);    // dQ = dS K
-      const int ksteps = a.D / 16;
-      bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma);
+      // dQ: with a 128-wide head dim the transposed product dQ^T = K^T dS^T
+      // (TMEM lane = head-dim index, column = query) lets the drain add whole
+      // 128-byte rows; otherwise dQ = dS K (lane = query).
+      const uint32_t idesc_dq = C::kDqTransposed ? make_idesc(BF16, 128, 128, true, true)
+                                                 : make_idesc(BF16, 128, a.D, true, true);
+      // Descriptor words: the high word is fixed per layout; the low word
+      // carries the start address and is advanced by (bytes >> 4).
+      const uint32_t hiK = (uint32_t)(make_sdesc(0, 16, 1024) >> 32);    // K-major
+      const uint32_t hiM = (uint32_t)(make_sdesc(0, 16384, 1024) >> 32); // MN-major
+      const uint32_t loK = (uint32_t)make_sdesc(sK, 16, 1024), loV = (uint32_t)make_sdesc(sV, 16, 1024);
+      const uint32_t loQ = (uint32_t)make_sdesc(sQ, 16, 1024), loDO = (uint32_t)make_sdesc(sDO, 16, 1024);
+      const uint32_t loKm = (uint32_t)make_sdesc(sK, 16384, 1024);
+      const uint32_t loQm = (uint32_t)make_sdesc(sQ, 16384, 1024);
+      const uint32_t loDOm = (uint32_t)make_sdesc(sDO, 16384, 1024);
+      const uint32_t loDSm = (uint32_t)make_sdesc(sDS, 16384, 1024);
+      constexpr uint32_t kTile16 = C::kTileBytes >> 4;
+      bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma) &&
+                mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma);
+      if (ok) {
+        tc_fence_after();
+        bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ, hiK, idesc_kk);
+        tc_commit(s_full);
+        ok = mbar_wait(do_full(0), 0, abort_flag, a.status, kSiteMma);
+      }
+      if (ok) {
+        tc_fence_after();
+        bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO, hiK, idesc_kk);
+        tc_commit(dp_full);
+      }
       for (int it = 0; it < n_it && ok; ++it) {
         const int qs = it % C::kQStages;
-        const uint32_t par = (it / C::kQStages) & 1;
-        const uint32_t qb = sQ + qs * C::kTileBytes, dob = sDO + qs * C::kTileBytes;
-        if (!(ok = mbar_wait(q_full(qs), par, abort_flag, a.status, kSiteMma))) break;
-        tc_fence_after();
-        for (int kk = 0; kk < ksteps; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::kColS, make_sdesc(sK + off, 16, 1024), make_sdesc(qb + off, 16, 1024),
-                 idesc_kk, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(s_full);
-        if (!(ok = mbar_wait(do_full(qs), par, abort_flag, a.status, kSiteMma))) break;
-        if (C::kAliasDQ && it > 0 &&
-            !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag, a.status, kSiteMma)))
-          break;
-        tc_fence_after();
-        for (int kk = 0; kk < ksteps; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::kColDP, make_sdesc(sV + off, 16, 1024), make_sdesc(dob + off, 16, 1024),
-                 idesc_kk, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(dp_full);
+        const int nx = it + 1, nqs = nx % C::kQStages;
+        const uint32_t npar = (nx / C::kQStages) & 1;
+        // dV += P^T dO  (P^T from TMEM, dO MN-major)
         if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
         tc_fence_after();
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(tmem + C::kColDV, tmem + C::kColS + 8 * kk, make_sdesc(dob + kk * 2048, 16384, 1024),
-                 idesc_acc, acc);
-          mma_ts(tmem + C::kColDK, tmem + C::kColDP + 8 * kk, make_sdesc(qb + kk * 2048, 16384, 1024),
-                 idesc_acc, acc);
-        }
-        tc_commit(q_empty(qs));
+        bwd_issue_ts(tmem + C::kColDV, tmem + C::kColS, loDOm + qs * kTile16, hiM, idesc_acc, it > 0);
         tc_commit(do_empty(qs));
+        if (nx < n_it) {
+          if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
+          tc_fence_after();
+          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ + nqs * kTile16, hiK, idesc_kk);
+          tc_commit(s_full);
+        }
+        // dK += dS^T Q
+        if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
+        tc_fence_after();
+        bwd_issue_ts(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_acc, it > 0);
+        tc_commit(q_empty(qs));
+        // dQ tile (into the dP columns when aliased: in order after dK read them)
         if (!C::kAliasDQ && it > 0 &&
             !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag, a.status, kSiteMma)))
           break;
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + C::kColDQ, make_sdesc(sDS + kk * 2048, 16384, 1024),
-                 make_sdesc(sK + kk * 2048, 16384, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+        if (C::kDqTransposed)
+          bwd_issue_mn(tmem + C::kColDQ, loKm, loDSm, hiM, idesc_dq);   // K^T dS^T
+        else
+          bwd_issue_mn(tmem + C::kColDQ, loDSm, loKm, hiM, idesc_dq);   // dS K
         tc_commit(dq_mma);
+        if (nx < n_it) {
+          if (!(ok = mbar_wait(do_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
+          if (C::kAliasDQ && !(ok = mbar_wait(dq_free, it & 1, abort_flag, a.status, kSiteMma)))
+            break;
+          tc_fence_after();
+          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + nqs * kTile16, hiK, idesc_kk);
+          tc_commit(dp_full);
+        }
       }
       tc_commit(acc_done);
     }
@@ -348,33 +405,54 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       const int32_t m0 = (mb + it) * 128;
       const bool full = tile_is_full(win, sq, sk, m0, n0);
       const int32_t ca = qa - m0, cz = qz - m0;  // allowed columns [ca, cz]
-      ok = mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
-           mbar_wait(dp_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
+      // ---- phase 1: P^T = exp2(S^T * c*log2(e) - LSE*log2(e)), masked ----
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax));
+      if (!ok) continue;
+      tc_fence_after();
+      // P is kept as the rounded 16-bit pairs the dV product uses (64 registers).
+      uint32_t pk[64];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sr[64];
+        tmem_ld64(tS + 64 * h2, sr);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int q0 = 64 * h2 + 2 * e, q1 = q0 + 1;
+          float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lse_s[q0]));
+          float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lse_s[q1]));
+          if (!full) {
+            v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
+            v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
+          }
+          pk[32 * h2 + e] = pack2<BF16>(v0, v1);
+        }
+        uint32_t chunk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) chunk[e] = pk[32 * h2 + e];
+        tmem_st32(tS + 32 * h2, chunk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      // ---- phase 2: dS^T = P^T o (dP^T - delta), into TMEM and shared memory ----
+      ok = mbar_wait(dp_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
            (it == 0 || mbar_wait(dq_mma, (it - 1) & 1, abort_flag, a.status, kSiteSoftmax));
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tS + 32 * c, sr);
-        tmem_ld32(tDP + 32 * c, dr);
-        uint32_t pp[16], dd[16];
+        uint32_t dr[32];
+        tmem_ld32(tDP + 32 * c, dr);  // chunk c of dP^T (32 queries)
+        uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int q0 = 32 * c + 2 * e, q1 = q0 + 1;
-          float p0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lse_s[q0]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lse_s[q1]));
-          if (!full) {
-            p0 = (q0 < ca || q0 > cz) ? 0.f : p0;
-            p1 = (q1 < ca || q1 > cz) ? 0.f : p1;
-          }
-          const float d0 = p0 * (__uint_as_float(dr[2 * e]) - dl_s[q0]);
-          const float d1 = p1 * (__uint_as_float(dr[2 * e + 1]) - dl_s[q1]);
-          pp[e] = pack2<BF16>(p0, p1);
+          const float2 pe = unpack2<BF16>(pk[16 * c + e]);
+          const float d0 = pe.x * (__uint_as_float(dr[2 * e]) - dl_s[q0]);
+          const float d1 = pe.y * (__uint_as_float(dr[2 * e + 1]) - dl_s[q1]);
           dd[e] = pack2<BF16>(d0, d1);
         }
-        tmem_st16(tS + 16 * c, pp);
         tmem_st16(tDP + 16 * c, dd);
         // dS (query-contiguous rows of this key) into the MN-major smem tile.
         const uint32_t rowb = sDS + (c >> 1) * 16384 + r * 128;
@@ -389,7 +467,7 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive(ds_ready);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, a.status, kSiteEpilogue));
     if (ok) {
@@ -418,24 +496,43 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
   } else {
     // ===================== dQ drain (warps 4-7) =====================
     const int quad = warp & 3;
-    const int q = quad * 32 + lane;  // query row within the tile
+    const int t = quad * 32 + lane;  // TMEM lane of this thread
     const uint32_t tDQ = tmem + ((uint32_t)(quad * 32) << 16) + C::kColDQ;
     for (int it = 0; it < n_it; ++it) {
       bool ok = mbar_wait(dq_mma, it & 1, abort_flag, a.status, kSiteDq);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int32_t i = (mb + it) * 128 + q;
-      const bool valid = i < sq;
-      const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
-      float* dst = a.dq_acc + ((int64_t)h * a.rows + row) * a.D;
-      for (int c = 0; c < a.D / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(tDQ + 16 * c, v);
-        if (valid) {
+      const int32_t m0 = (mb + it) * 128;
+      const int64_t row0 = a.packed ? (int64_t)(qrow0 + m0) : (int64_t)b * a.Sq + m0;
+      float* base = a.dq_acc + ((int64_t)h * a.rows + row0) * a.D;
+      if (C::kDqTransposed) {
+        // lane t = head-dim index d, column = query: a warp adds 32 consecutive
+        // floats of one query row per instruction.  The whole tile is pulled
+        // into registers first and the TMEM columns released before the
+        // reductions are issued, so the next MMA into them need not wait.
+        const int nq = min(128, sq - m0);
+        uint32_t v[128];
+        tmem_ld128(tDQ, v);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        if (t < a.D) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            red_add_v4(dst + 16 * c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          for (int q = 0; q < 128; ++q)
+            if (q < nq) red_add_f32(base + (int64_t)q * a.D + t, __uint_as_float(v[q]));
+        }
+        continue;
+      } else {
+        const bool valid = m0 + t < sq;
+        float* dst = base + (int64_t)t * a.D;
+        for (int c = 0; c < a.D / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16(tDQ + 16 * c, v);
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              red_add_v4(dst + 16 * c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                         __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
         }
       }
       tc_fence_before();

@@ -27,10 +27,18 @@ struct FwdCfg {
   static constexpr int kSoftmaxWarps = 4 * NQ;
   static constexpr int kLoadWarp = kSoftmaxWarps;
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  // One more full warpgroup after the softmax groups (TMA warp, MMA warp and
+  // two spare warps), so registers can be moved between warpgroups.
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
+  // Register split (setmaxnreg): the launch gives every thread kLaunchRegs;
+  // the producer/MMA group drops to kLowRegs, the softmax groups rise to
+  // kHighRegs.  NQ*128*kHighRegs + 128*kLowRegs == kThreads*kLaunchRegs.
+  static constexpr int kLaunchRegs = 168;  // 65536 / (4 sub-partitions x 3 warps x 32) rounded to 8
+  static constexpr int kLowRegs = 136;
+  static constexpr int kHighRegs = (kThreads * kLaunchRegs - 128 * kLowRegs) / (128 * NQ) / 8 * 8;
   static constexpr int kBlocks = DPAD / 64;                // 128-byte swizzle blocks per row
   static constexpr int kTileBytes = 128 * DPAD * 2;        // one 128-row tile of Q, K or V
-  static constexpr int kKStages = DPAD == 128 ? 2 : 4;
+  static constexpr int kKStages = DPAD == 128 ? 3 : 4;
   static constexpr int kVStages = DPAD == 128 ? 2 : 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + NQ * kTileBytes;
@@ -44,6 +52,29 @@ struct FwdCfg {
   static constexpr int kTmemCols = (128 * NQ + DPAD * NQ) <= 256 ? 256 : 512;
   static constexpr int kColO = 128 * NQ;
 };
+
+// O (+)= P V for one query tile: P from TMEM (8 columns per K step of 16
+// keys), V MN-major in shared memory (next 16 keys = +2048 bytes).
+__device__ __forceinline__ void fwd_issue_pv(uint32_t d, uint32_t a, uint32_t vd, uint32_t hi,
+                                             uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts2(d, a + 8 * kk, vd + (uint32_t)(kk * 2048 >> 4), hi, idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// S = Q K^T for one query tile: both K-major; 16-column K steps are +32 bytes
+// inside a 64-column block, blocks 16 KiB apart.  Padded head-dim columns
+// are zero in both operands (TMA fill), so all KSTEPS steps are issued.
+template <int KSTEPS>
+__device__ __forceinline__ void fwd_issue_s(uint32_t d, uint32_t qd, uint32_t kd, uint32_t hi,
+                                            uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk) {
+    const uint32_t o = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+    mma_ss2(d, qd + o, hi, kd + o, hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
 
 template <int NQ, int DPAD, bool BF16>
 __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
@@ -152,6 +183,9 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= C::kSoftmaxWarps) {
+  // The producer / MMA warpgroup gives registers back to the softmax groups.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kLowRegs));
   if (warp == C::kLoadWarp) {
     // ===================== TMA producer =====================
     if (lane == 0) {
@@ -198,24 +232,35 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
     }
   } else if (warp == C::kMmaWarp) {
     // ===================== MMA issuer =====================
+    // Shared-memory descriptors are built once per tile and advanced by adding
+    // (byte offset >> 4) to their start-address field, so issuing an MMA
+    // costs a 64-bit add, not a rebuilt descriptor.
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc(BF16, 128, 128, false, false, args.negate != 0);
       const uint32_t idesc_o = make_idesc(BF16, 128, args.D, false, true);
-      const int ksteps = args.D / 16;
+      // descriptor words: hi is fixed per layout, lo carries the start address
+      const uint32_t kHiK = (uint32_t)(make_sdesc(0, 16, 1024) >> 32);
+      const uint32_t kHiV = (uint32_t)(make_sdesc(0, 16384, 1024) >> 32);
+      const uint32_t dQ = (uint32_t)make_sdesc(sQ, 16, 1024), dK = (uint32_t)make_sdesc(sK, 16, 1024);
+      const uint32_t dV = (uint32_t)make_sdesc(sV, 16384, 1024);
+      constexpr uint32_t kTile16 = C::kTileBytes >> 4;
       bool ok = true;
       for (int t = 0; t < NQ && ok; ++t)
         ok = mbar_wait(q_full(t), 0, abort_flag, args.status, kSiteMma);
-      auto issue_pv = [&](int t, int it_prev) {
-        const int vs = it_prev % C::kVStages;
-        const uint32_t vbase = sV + vs * C::kTileBytes;
-        for (int kk = 0; kk < 8; ++kk) {
-          // B = V tile, MN-major: 64-column blocks 16 KiB apart, K step of 16
-          // key rows = 2048 bytes.
-          const uint64_t bdesc = make_sdesc(vbase + kk * 2048, 16384, 1024);
-          mma_ts(tmem + C::kColO + DPAD * t, tmem + 128 * t + kk * 8, bdesc, idesc_o,
-                 (it_prev > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(o_done(t));
+      // O_t (+)= P_t V: P from TMEM (16 columns of 32 bits per 16 keys... 8
+      // columns per K step of 16 keys), V MN-major, next 16 keys = +2048 bytes.
+      auto issue_pv = [=](int t, int it_prev) {
+        fwd_issue_pv(tmem + C::kColO + DPAD * t, tmem + 128 * t,
+                     dV + (uint32_t)(it_prev % C::kVStages) * kTile16, kHiV, idesc_o, it_prev > 0);
+        tc_commit(bar0 + 8 * (bs + 2 * NQ + t));  // o_done(t)
+      };
+      // S_t = Q_t K^T: both K-major; 16-column K steps are +32 bytes inside a
+      // 64-column block, blocks 16 KiB apart.  Padded head-dim columns are
+      // zero in both operands (TMA fill), so all DPAD/16 steps are issued.
+      auto issue_s = [=](int t, int ks) {
+        fwd_issue_s<DPAD / 16>(tmem + 128 * t, dQ + (uint32_t)t * kTile16,
+                               dK + (uint32_t)ks * kTile16, kHiK, idesc_s);
+        tc_commit(bar0 + 8 * (bs + t));  // s_full(t)
       };
       for (int it = 0; it < n_tiles && ok; ++it) {
         const int ks = it % C::kKStages;
@@ -232,20 +277,12 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
             }
             tc_fence_after();
             issue_pv(t, it - 1);
+            if (t == NQ - 1) tc_commit(v_empty((it - 1) % C::kVStages));
           }
-          // S_t = Q_t K^T: both K-major, 16-column K steps inside 64-column
-          // blocks (+32 bytes), next block at +16 KiB.
-          const uint32_t qbase = sQ + t * C::kTileBytes, kbase = sK + ks * C::kTileBytes;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + 128 * t, make_sdesc(qbase + off, 16, 1024),
-                   make_sdesc(kbase + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(s_full(t));
+          issue_s(t, ks);
         }
         if (!ok) break;
         tc_commit(k_empty(ks));
-        if (it > 0) tc_commit(v_empty((it - 1) % C::kVStages));
       }
       if (ok) {
         const int last = n_tiles - 1;
@@ -265,7 +302,9 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, args.status, kSiteTeardown);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kHighRegs));
     // ===================== softmax / correction / epilogue =====================
     const int t = warp / 4;               // query tile of this warp group
     const int quad = warp % 4;            // TMEM lane quadrant
@@ -282,14 +321,12 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       ok = mbar_wait(s_full(t), it & 1, abort_flag, args.status, kSiteSoftmax);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
+      // The whole score row in one TMEM load.
+      uint32_t raw[128];
+      tmem_ld128(tS, raw);
       float s[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tS + 32 * c, raw);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(raw[e]);
-      }
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c]);
       const int32_t n0 = (nb + it) * 128;
       const bool full = tile_is_full(win, sq, sk, m0 + 128 * t, n0);
       if (!full) {
@@ -298,9 +335,14 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c < a || c > z) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      // Row maximum over 8 independent chains (short dependency chains).
+      float m8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int k = 0; k < 8; ++k) m8[k] = s[k];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2;
       // Lazy rescale: keep the running reference unless the new maximum
       // exceeds it by more than 2^8 (P stays below 256, exact in fp32 sums).
@@ -310,7 +352,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         m_used = m_tile;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float rowsum = 0.f;
+      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t packed[16];
@@ -322,11 +364,12 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
             p0 = (x0 == -INFINITY) ? 0.f : p0;
             p1 = (x1 == -INFINITY) ? 0.f : p1;
           }
-          rowsum += p0 + p1;
+          l8[e & 7] += p0 + p1;
           packed[e] = pack2<BF16>(p0, p1);
         }
         tmem_st16(tS + 16 * c, packed);
       }
+      const float rowsum = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       l = alpha * l + rowsum;
       if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O_t must hold PV of the previous tile before it is rescaled.
@@ -384,9 +427,17 @@ template <int NQ, int DPAD, bool BF16>
 static cudaError_t launch(const FwdArgs& args, int n_mblocks, cudaStream_t stream) {
   using C = FwdCfg<NQ, DPAD>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  static_assert(NQ * 128 * C::kHighRegs + 128 * C::kLowRegs <= C::kThreads * C::kLaunchRegs,
+                "register split exceeds the launch budget");
   auto kern = attn_fwd_kernel<NQ, DPAD, BF16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  // The setmaxnreg split assumes every thread starts with kLaunchRegs
+  // registers; with fewer, the raising warpgroups would wait forever, so
+  // refuse to launch instead.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < C::kLaunchRegs) return cudaErrorLaunchOutOfResources;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(n_mblocks, args.H, args.B);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(args);
