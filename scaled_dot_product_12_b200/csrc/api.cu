@@ -152,6 +152,21 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 2-D fp32 map over the dQ accumulator [H*rows][D] (row pitch D*4 bytes),
+// 32 x 32 boxes, no swizzle: the backward adds staged dQ tiles through it.
+cudaError_t make_dq_map(CUtensorMap* map, float* base, int D, int64_t rows_total) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(rows_total > 0 ? rows_total : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Checks shared by forward and backward.
 template <class P>
 bool common_ok(const P* p, size_t want_size, Mode* m, bool check_pointers = true) {
@@ -309,6 +324,8 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     const size_t delta_bytes = ((size_t)p->H * rows_q * 4 + 255) & ~(size_t)255;
     a.delta = static_cast<float*>(p->workspace);
     a.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(p->workspace) + delta_bytes);
+    e = make_dq_map(&a.tdq, a.dq_acc, p->D, (int64_t)p->H * rows_q);
+    if (e != cudaSuccess) return e;
     a.status = info.status;
     a.main_events[0] = static_cast<cudaEvent_t>(p->main_kernel_events[0]);
     a.main_events[1] = static_cast<cudaEvent_t>(p->main_kernel_events[1]);

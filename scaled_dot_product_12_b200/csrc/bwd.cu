@@ -104,16 +104,23 @@ struct BwdCfg {
   static constexpr int kBlocks = DPAD / 64;
   static constexpr int kTileBytes = 128 * DPAD * 2;
   static constexpr int kQStages = 2;
+  // dQ^T path (head dim 128): the dQ tile is staged in shared memory for TMA
+  // bulk reductions (4 warps x 2 buffers x 32x32 fp32); dO gets one ring
+  // stage to make room.
+  static constexpr bool kStageDq = (DPAD == 128);
+  static constexpr int kDOStages = kStageDq ? 1 : 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;
   static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
-  static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;  // 128 x 128 16-bit
-  static constexpr int kOffRow = kOffDS + 128 * 128 * 2;          // lse/delta [2][2][128] f32
+  static constexpr int kOffDS = kOffDO + kDOStages * kTileBytes;  // 128 x 128 16-bit
+  static constexpr int kOffDQ = kOffDS + 128 * 128 * 2;
+  static constexpr int kDqStageBytes = kStageDq ? 4 * 2 * 32 * 32 * 4 : 0;
+  static constexpr int kOffRow = kOffDQ + kDqStageBytes;           // lse/delta [2][2][128] f32
   static constexpr int kOffBar = kOffRow + 2 * 2 * 128 * 4;
-  // kv_full, q_full[QS], q_empty[QS], do_full[QS], do_empty[QS], s_full,
+  // kv_full, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
   // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done
-  static constexpr int kNumBars = 1 + 4 * kQStages + 7;
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 7;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + DPAD;
@@ -202,15 +209,15 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
   }
 
   const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV, sQ = sbase + C::kOffQ,
-                 sDO = sbase + C::kOffDO, sDS = sbase + C::kOffDS;
+                 sDO = sbase + C::kOffDO, sDS = sbase + C::kOffDS, sDQ = sbase + C::kOffDQ;
   float* row_s = reinterpret_cast<float*>(smem + C::kOffRow);  // [buf][lse|delta][128]
   const uint32_t bar0 = sbase + C::kOffBar;
   const uint32_t kv_full = bar0;
   auto q_full = [&](int s) { return bar0 + 8 * (1 + s); };
   auto q_empty = [&](int s) { return bar0 + 8 * (1 + C::kQStages + s); };
   auto do_full = [&](int s) { return bar0 + 8 * (1 + 2 * C::kQStages + s); };
-  auto do_empty = [&](int s) { return bar0 + 8 * (1 + 3 * C::kQStages + s); };
-  const uint32_t s_full = bar0 + 8 * (1 + 4 * C::kQStages);
+  auto do_empty = [&](int s) { return bar0 + 8 * (1 + 2 * C::kQStages + C::kDOStages + s); };
+  const uint32_t s_full = bar0 + 8 * (1 + 2 * C::kQStages + 2 * C::kDOStages);
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24,
                  dq_mma = s_full + 32, dq_free = s_full + 40, acc_done = s_full + 48;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -221,6 +228,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
     for (int s = 0; s < C::kQStages; ++s) {
       mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), 1);
+    }
+    for (int s = 0; s < C::kDOStages; ++s) {
       mbar_init(do_full(s), 1);
       mbar_init(do_empty(s), 1);
     }
@@ -266,11 +275,13 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
           tma_load_4d(sQ + qs * C::kTileBytes + blk * 16384, &a.tq, q_full(qs), 64 * blk, qrow, h,
                       bcoord);
         ++nq;
-        if (round > 0 && !mbar_wait(do_empty(qs), (round - 1) & 1, abort_flag, a.status, kSiteLoad))
+        const int ds = it % C::kDOStages, dround = it / C::kDOStages;
+        if (dround > 0 &&
+            !mbar_wait(do_empty(ds), (dround - 1) & 1, abort_flag, a.status, kSiteLoad))
           break;
-        mbar_expect_tx(do_full(qs), C::kTileBytes);
+        mbar_expect_tx(do_full(ds), C::kTileBytes);
         for (int blk = 0; blk < C::kBlocks; ++blk)
-          tma_load_4d(sDO + qs * C::kTileBytes + blk * 16384, &a.tdo, do_full(qs), 64 * blk, qrow,
+          tma_load_4d(sDO + ds * C::kTileBytes + blk * 16384, &a.tdo, do_full(ds), 64 * blk, qrow,
                       h, bcoord);
         ++ndo;
       }
@@ -279,8 +290,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
         for (int it = max(0, nq - C::kQStages); it < nq; ++it)
           mbar_wait(q_full(it % C::kQStages), (it / C::kQStages) & 1, abort_flag, a.status,
                     kSiteTeardown);
-        for (int it = max(0, ndo - C::kQStages); it < ndo; ++it)
-          mbar_wait(do_full(it % C::kQStages), (it / C::kQStages) & 1, abort_flag, a.status,
+        for (int it = max(0, ndo - C::kDOStages); it < ndo; ++it)
+          mbar_wait(do_full(it % C::kDOStages), (it / C::kDOStages) & 1, abort_flag, a.status,
                     kSiteTeardown);
       }
     }
@@ -322,14 +333,14 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
         tc_commit(dp_full);
       }
       for (int it = 0; it < n_it && ok; ++it) {
-        const int qs = it % C::kQStages;
-        const int nx = it + 1, nqs = nx % C::kQStages;
-        const uint32_t npar = (nx / C::kQStages) & 1;
+        const int qs = it % C::kQStages, dos = it % C::kDOStages;
+        const int nx = it + 1, nqs = nx % C::kQStages, ndos = nx % C::kDOStages;
+        const uint32_t npar = (nx / C::kQStages) & 1, ndpar = (nx / C::kDOStages) & 1;
         // dV += P^T dO  (P^T from TMEM, dO MN-major)
         if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
         tc_fence_after();
-        bwd_issue_ts(tmem + C::kColDV, tmem + C::kColS, loDOm + qs * kTile16, hiM, idesc_acc, it > 0);
-        tc_commit(do_empty(qs));
+        bwd_issue_ts(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_acc, it > 0);
+        tc_commit(do_empty(dos));
         if (nx < n_it) {
           if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
           tc_fence_after();
@@ -351,11 +362,11 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
           bwd_issue_mn(tmem + C::kColDQ, loDSm, loKm, hiM, idesc_dq);   // dS K
         tc_commit(dq_mma);
         if (nx < n_it) {
-          if (!(ok = mbar_wait(do_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
+          if (!(ok = mbar_wait(do_full(ndos), ndpar, abort_flag, a.status, kSiteMma))) break;
           if (C::kAliasDQ && !(ok = mbar_wait(dq_free, it & 1, abort_flag, a.status, kSiteMma)))
             break;
           tc_fence_after();
-          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + nqs * kTile16, hiK, idesc_kk);
+          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + ndos * kTile16, hiK, idesc_kk);
           tc_commit(dp_full);
         }
       }
@@ -415,11 +426,17 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t sr[64];
         tmem_ld64(tS + 64 * h2, sr);
+        float lv[64];  // LSE*log2(e) of these 64 queries, read 4 at a time
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float4 t4 = reinterpret_cast<const float4*>(lse_s)[16 * h2 + j];
+          lv[4 * j] = t4.x; lv[4 * j + 1] = t4.y; lv[4 * j + 2] = t4.z; lv[4 * j + 3] = t4.w;
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int q0 = 64 * h2 + 2 * e, q1 = q0 + 1;
-          float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lse_s[q0]));
-          float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lse_s[q1]));
+          float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lv[2 * e]));
+          float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lv[2 * e + 1]));
           if (!full) {
             v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
             v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
@@ -444,13 +461,18 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       for (int c = 0; c < 4; ++c) {
         uint32_t dr[32];
         tmem_ld32(tDP + 32 * c, dr);  // chunk c of dP^T (32 queries)
+        float dv[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 t4 = reinterpret_cast<const float4*>(dl_s)[8 * c + j];
+          dv[4 * j] = t4.x; dv[4 * j + 1] = t4.y; dv[4 * j + 2] = t4.z; dv[4 * j + 3] = t4.w;
+        }
         uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int q0 = 32 * c + 2 * e, q1 = q0 + 1;
           const float2 pe = unpack2<BF16>(pk[16 * c + e]);
-          const float d0 = pe.x * (__uint_as_float(dr[2 * e]) - dl_s[q0]);
-          const float d1 = pe.y * (__uint_as_float(dr[2 * e + 1]) - dl_s[q1]);
+          const float d0 = pe.x * (__uint_as_float(dr[2 * e]) - dv[2 * e]);
+          const float d1 = pe.y * (__uint_as_float(dr[2 * e + 1]) - dv[2 * e + 1]);
           dd[e] = pack2<BF16>(d0, d1);
         }
         tmem_st16(tDP + 16 * c, dd);
@@ -510,16 +532,34 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
         // floats of one query row per instruction.  The whole tile is pulled
         // into registers first and the TMEM columns released before the
         // reductions are issued, so the next MMA into them need not wait.
-        const int nq = min(128, sq - m0);
         uint32_t v[128];
         tmem_ld128(tDQ, v);
         tc_fence_before();
         mbar_arrive(dq_free);
-        if (t < a.D) {
+        // Stage 32 x 32 boxes (query rows x this warp's 32 head-dim columns)
+        // and add them into the accumulator with TMA bulk reductions; rows of
+        // queries outside the sequence hold exact zeros (their dS is 0).
+        if (32 * quad < a.D) {
+          const uint32_t stage = sDQ + quad * 8192;
+          const int grow = (int)((int64_t)h * a.rows + row0);
 #pragma unroll
-          for (int q = 0; q < 128; ++q)
-            if (q < nq) red_add_f32(base + (int64_t)q * a.D + t, __uint_as_float(v[q]));
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t buf = stage + (c & 1) * 4096;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + e * 128 + lane * 4), "r"(v[32 * c + e])
+                           : "memory");
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_2d(&a.tdq, buf, 32 * quad, grow + 32 * c);
+              bulk_commit();
+            }
+          }
         }
+        (void)base;
         continue;
       } else {
         const bool valid = m0 + t < sq;
@@ -538,6 +578,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       tc_fence_before();
       mbar_arrive(dq_free);
     }
+    // The staged tiles must stay in place until the TMA has added them.
+    if (C::kStageDq && lane == 0) bulk_wait<0>();
   }
 
   __syncwarp();

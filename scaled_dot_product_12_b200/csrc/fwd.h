@@ -26,6 +26,7 @@ struct FwdArgs {
 
 struct BwdArgs {
   CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tdq;  // fp32 dQ accumulator as 2-D (D, H*rows), 32 x 32 boxes
   const void* o;
   const void* dout;
   const float* lse;
