@@ -16,8 +16,8 @@
 //                           notes, "Kernel Bug Fixes", record a kernel that
 //                           addressed dO with O's strides);
 //  3. attn_dq_convert_kernel  dQ = sm_scale * accumulator in the input dtype.
-// Warp roles of (2): warps 0-3 "ds" (one key row per thread: P, dS, epilogue),
-// warps 4-7 dQ drain (one query row per thread), warp 8 TMA, warp 9 MMA.
+// Warp roles of (2): warps 0-7 P / dS in two groups of query columns (one key
+// row per thread), warps 8-11 dQ drain, warp 12 TMA, warp 13 MMA.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -98,9 +98,12 @@ __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_const
 // ---------------------------------------------------------------------------
 template <int DPAD>
 struct BwdCfg {
-  static constexpr int kThreads = 320;
-  static constexpr int kLoadWarp = 8;
-  static constexpr int kMmaWarp = 9;
+  // Warps 0-7: two P/dS groups (query columns 0-63 and 64-127 of every key
+  // row); 8-11: dQ drain; 12: TMA; 13: MMA.  14 warps: at most 4 per
+  // sub-partition, so 128 registers per thread.
+  static constexpr int kThreads = 448;
+  static constexpr int kLoadWarp = 12;
+  static constexpr int kMmaWarp = 13;
   static constexpr int kBlocks = DPAD / 64;
   static constexpr int kTileBytes = 128 * DPAD * 2;
   static constexpr int kQStages = 2;
@@ -150,6 +153,15 @@ __device__ __forceinline__ void bwd_issue_ts(uint32_t d, uint32_t a, uint32_t b_
     mma_ts2(d, a + 8 * kk, b_lo + (uint32_t)(kk * 2048 >> 4), hi, idesc,
             (accumulate || kk > 0) ? 1u : 0u);
 }
+// Same with A split in two: queries 0-63 at columns [a, a+32), queries
+// 64-127 at [a+64, a+96) (each P/dS group writes inside its own columns).
+__device__ __forceinline__ void bwd_issue_ts_halves(uint32_t d, uint32_t a, uint32_t b_lo,
+                                                    uint32_t hi, uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts2(d, a + 8 * kk + (kk >= 4 ? 32 : 0), b_lo + (uint32_t)(kk * 2048 >> 4), hi, idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
 // D = A B with both operands MN-major in smem, K = 128 (16 rows = 2048 bytes).
 __device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
                                              uint32_t idesc) {
@@ -161,7 +173,7 @@ __device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t
 }
 
 template <int DPAD, bool BF16>
-__global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<DPAD>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -235,8 +247,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_ready, 128);
-    mbar_init(ds_ready, 128);
+    mbar_init(p_ready, 256);
+    mbar_init(ds_ready, 256);
     mbar_init(dq_mma, 1);
     mbar_init(dq_free, 128);
     mbar_init(acc_done, 1);
@@ -252,6 +264,7 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 12) {
   if (warp == C::kLoadWarp) {
     // ===================== TMA producer =====================
     if (lane == 0) {
@@ -339,7 +352,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
         // dV += P^T dO  (P^T from TMEM, dO MN-major)
         if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
         tc_fence_after();
-        bwd_issue_ts(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_acc, it > 0);
+        bwd_issue_ts_halves(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_acc,
+                            it > 0);
         tc_commit(do_empty(dos));
         if (nx < n_it) {
           if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
@@ -350,7 +364,8 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
         // dK += dS^T Q
         if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
         tc_fence_after();
-        bwd_issue_ts(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_acc, it > 0);
+        bwd_issue_ts_halves(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_acc,
+                            it > 0);
         tc_commit(q_empty(qs));
         // dQ tile (into the dP columns when aliased: in order after dK read them)
         if (!C::kAliasDQ && it > 0 &&
@@ -372,47 +387,51 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       }
       tc_commit(acc_done);
     }
-  } else if (warp < 4) {
+  }
+  } else if (warp < 8) {
     // ===================== P, dS and the dK / dV epilogue =====================
-    const int r = warp * 32 + lane;  // key row within the tile
+    // Group `half` owns query columns [64 half, 64 half + 64) of every key row.
+    const int half = warp >> 2, quad = warp & 3;
+    const int r = quad * 32 + lane;  // key row within the tile (TMEM lane)
     const int32_t j = n0 + r;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
+    const int qo = 64 * half;          // first query column of this group
+    const uint32_t po = 64 * half;     // its P / dS columns (16-bit pairs)
     const float sl2 = a.scale_log2;
     // Queries that see key j: j - R <= i <= j + L, 0 <= i < sq (none if j >= sk).
     int32_t qa = j - win.R, qz = j + win.L;
     if (qa < 0) qa = 0;
     if (qz > sq - 1) qz = sq - 1;
     if (j >= sk) qz = qa - 1;
-    auto row_vals = [&](int it, float& lse, float& dl) {
+    // Per-query values of a tile, one per thread: group 0 fetches LSE*log2(e),
+    // group 1 fetches delta, for query row r.
+    auto row_val = [&](int it) -> float {
       const int32_t i = (mb + it) * 128 + r;
-      lse = 0.f;
-      dl = 0.f;
-      if (i < sq) {
+      if (i >= sq) return 0.f;
+      if (half == 0) {
         int64_t li;
         if (a.packed)
           li = a.lse_th ? (int64_t)(qrow0 + i) * a.H + h : (int64_t)h * a.total_q + qrow0 + i;
         else
           li = a.lse_th ? ((int64_t)b * a.Sq + i) * a.H + h : ((int64_t)b * a.H + h) * a.Sq + i;
-        lse = a.lse[li] * 1.4426950408889634f;
-        const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
-        dl = a.delta[(int64_t)h * a.rows + row];
+        return a.lse[li] * 1.4426950408889634f;
       }
+      const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
+      return a.delta[(int64_t)h * a.rows + row];
     };
-    float lse_n, dl_n;
-    row_vals(0, lse_n, dl_n);
+    float val_n = row_val(0);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int buf = it & 1;
       float* lse_s = row_s + buf * 256;
       float* dl_s = lse_s + 128;
-      lse_s[r] = lse_n;
-      dl_s[r] = dl_n;
-      // Every warp of the group passes this barrier once per tile, aborted or
-      // not, so none can be left waiting at it.
-      named_bar_sync(1, 128);
+      (half == 0 ? lse_s : dl_s)[r] = val_n;
+      // Every warp of both groups passes this barrier once per tile, aborted
+      // or not, so none can be left waiting at it.
+      named_bar_sync(1, 256);
       if (!ok) continue;
-      if (it + 1 < n_it) row_vals(it + 1, lse_n, dl_n);
+      if (it + 1 < n_it) val_n = row_val(it + 1);
       const int32_t m0 = (mb + it) * 128;
       const bool full = tile_is_full(win, sq, sk, m0, n0);
       const int32_t ca = qa - m0, cz = qz - m0;  // allowed columns [ca, cz]
@@ -420,33 +439,32 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax));
       if (!ok) continue;
       tc_fence_after();
-      // P is kept as the rounded 16-bit pairs the dV product uses (64 registers).
-      uint32_t pk[64];
+      // P is kept as the rounded 16-bit pairs the dV product uses.
+      uint32_t pk[32];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t sr[64];
-        tmem_ld64(tS + 64 * h2, sr);
-        float lv[64];  // LSE*log2(e) of these 64 queries, read 4 at a time
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(tS + qo + 32 * c, sr);
+        float lv[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float4 t4 = reinterpret_cast<const float4*>(lse_s)[16 * h2 + j];
-          lv[4 * j] = t4.x; lv[4 * j + 1] = t4.y; lv[4 * j + 2] = t4.z; lv[4 * j + 3] = t4.w;
+        for (int jj = 0; jj < 8; ++jj) {
+          const float4 t4 = reinterpret_cast<const float4*>(lse_s)[(qo >> 2) + 8 * c + jj];
+          lv[4 * jj] = t4.x; lv[4 * jj + 1] = t4.y; lv[4 * jj + 2] = t4.z; lv[4 * jj + 3] = t4.w;
         }
+        uint32_t chunk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q0 = 64 * h2 + 2 * e, q1 = q0 + 1;
+        for (int e = 0; e < 16; ++e) {
+          const int q0 = qo + 32 * c + 2 * e, q1 = q0 + 1;
           float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lv[2 * e]));
           float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lv[2 * e + 1]));
           if (!full) {
             v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
             v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
           }
-          pk[32 * h2 + e] = pack2<BF16>(v0, v1);
+          chunk[e] = pack2<BF16>(v0, v1);
+          pk[16 * c + e] = chunk[e];
         }
-        uint32_t chunk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) chunk[e] = pk[32 * h2 + e];
-        tmem_st32(tS + 32 * h2, chunk);
+        tmem_st16(tS + po + 16 * c, chunk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -458,14 +476,14 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
       if (!ok) continue;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
-        tmem_ld32(tDP + 32 * c, dr);  // chunk c of dP^T (32 queries)
+        tmem_ld32(tDP + qo + 32 * c, dr);  // 32 queries of dP^T
         float dv[32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 t4 = reinterpret_cast<const float4*>(dl_s)[8 * c + j];
-          dv[4 * j] = t4.x; dv[4 * j + 1] = t4.y; dv[4 * j + 2] = t4.z; dv[4 * j + 3] = t4.w;
+        for (int jj = 0; jj < 8; ++jj) {
+          const float4 t4 = reinterpret_cast<const float4*>(dl_s)[(qo >> 2) + 8 * c + jj];
+          dv[4 * jj] = t4.x; dv[4 * jj + 1] = t4.y; dv[4 * jj + 2] = t4.z; dv[4 * jj + 3] = t4.w;
         }
         uint32_t dd[16];
 #pragma unroll
@@ -475,12 +493,13 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
           const float d1 = pe.y * (__uint_as_float(dr[2 * e + 1]) - dv[2 * e + 1]);
           dd[e] = pack2<BF16>(d0, d1);
         }
-        tmem_st16(tDP + 16 * c, dd);
-        // dS (query-contiguous rows of this key) into the MN-major smem tile.
-        const uint32_t rowb = sDS + (c >> 1) * 16384 + r * 128;
+        tmem_st16(tDP + po + 16 * c, dd);
+        // dS (query-contiguous rows of this key) into the MN-major smem tile:
+        // 64-query block `half`, 16-byte chunks 4c..4c+3 of row r, swizzled.
+        const uint32_t rowb = sDS + half * 16384 + r * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int chunk = ((c & 1) * 4 + u) ^ (r & 7);
+          const int chunk = (c * 4 + u) ^ (r & 7);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + chunk * 16),
                        "r"(dd[4 * u]), "r"(dd[4 * u + 1]), "r"(dd[4 * u + 2]), "r"(dd[4 * u + 3])
                        : "memory");
@@ -493,30 +512,28 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, a.status, kSiteEpilogue));
     if (ok) {
+      // Group 0 stores dV, group 1 stores dK (scaled by sm_scale).
       tc_fence_after();
       const bool valid = j < sk;
-      uint8_t* dvrow = valid ? kv_row_ptr(a.dv, a.dv_stride, j) : nullptr;
-      uint8_t* dkrow = valid ? kv_row_ptr(a.dk, a.dk_stride, j) : nullptr;
+      uint8_t* row = valid ? (half == 0 ? kv_row_ptr(a.dv, a.dv_stride, j)
+                                        : kv_row_ptr(a.dk, a.dk_stride, j))
+                           : nullptr;
+      const float mul = half == 0 ? 1.f : a.sm_scale;
+      const uint32_t tacc = tmem + lane_off + (half == 0 ? C::kColDV : C::kColDK);
       for (int c = 0; c < a.D / 16; ++c) {
-        uint32_t rv[16], rk[16], pv[8], pk[8];
-        tmem_ld16(tmem + lane_off + C::kColDV + 16 * c, rv);
-        tmem_ld16(tmem + lane_off + C::kColDK + 16 * c, rk);
+        uint32_t rv[16], pv[8];
+        tmem_ld16(tacc + 16 * c, rv);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = pack2<BF16>(__uint_as_float(rv[2 * e]), __uint_as_float(rv[2 * e + 1]));
-          pk[e] = pack2<BF16>(__uint_as_float(rk[2 * e]) * a.sm_scale,
-                              __uint_as_float(rk[2 * e + 1]) * a.sm_scale);
-        }
+        for (int e = 0; e < 8; ++e)
+          pv[e] = pack2<BF16>(__uint_as_float(rv[2 * e]) * mul, __uint_as_float(rv[2 * e + 1]) * mul);
         if (valid) {
-          st_global_v4(dvrow + 32 * c, pv[0], pv[1], pv[2], pv[3]);
-          st_global_v4(dvrow + 32 * c + 16, pv[4], pv[5], pv[6], pv[7]);
-          st_global_v4(dkrow + 32 * c, pk[0], pk[1], pk[2], pk[3]);
-          st_global_v4(dkrow + 32 * c + 16, pk[4], pk[5], pk[6], pk[7]);
+          st_global_v4(row + 32 * c, pv[0], pv[1], pv[2], pv[3]);
+          st_global_v4(row + 32 * c + 16, pv[4], pv[5], pv[6], pv[7]);
         }
       }
     }
   } else {
-    // ===================== dQ drain (warps 4-7) =====================
+    // ===================== dQ drain (warps 8-11) =====================
     const int quad = warp & 3;
     const int t = quad * 32 + lane;  // TMEM lane of this thread
     const uint32_t tDQ = tmem + ((uint32_t)(quad * 32) << 16) + C::kColDQ;
@@ -532,31 +549,46 @@ __global__ void __launch_bounds__(320, 1) attn_bwd_kernel(const __grid_constant_
         // floats of one query row per instruction.  The whole tile is pulled
         // into registers first and the TMEM columns released before the
         // reductions are issued, so the next MMA into them need not wait.
-        uint32_t v[128];
-        tmem_ld128(tDQ, v);
-        tc_fence_before();
-        mbar_arrive(dq_free);
-        // Stage 32 x 32 boxes (query rows x this warp's 32 head-dim columns)
-        // and add them into the accumulator with TMA bulk reductions; rows of
-        // queries outside the sequence hold exact zeros (their dS is 0).
-        if (32 * quad < a.D) {
-          const uint32_t stage = sDQ + quad * 8192;
-          const int grow = (int)((int64_t)h * a.rows + row0);
+        // Two 64-query halves: the first half is staged before the second is
+        // read, then the TMEM columns are released and the second staged.
+        // Each 32-query chunk becomes a 32 x 32 box (query rows x this warp's
+        // head-dim columns) added by a TMA bulk reduction; rows of queries
+        // outside the sequence hold exact zeros (their dS is 0).
+        const bool active = 32 * quad < a.D;
+        const uint32_t stage = sDQ + quad * 8192;
+        const int grow = (int)((int64_t)h * a.rows + row0);
+        auto stage_chunk = [&](const uint32_t (&v)[64], int c) {
+          const uint32_t buf = stage + (c & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t buf = stage + (c & 1) * 4096;
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + e * 128 + lane * 4), "r"(v[32 * c + e])
-                           : "memory");
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_reduce_add_2d(&a.tdq, buf, 32 * quad, grow + 32 * c);
-              bulk_commit();
-            }
+          for (int e = 0; e < 32; ++e)
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + e * 128 + lane * 4),
+                         "r"(v[32 * (c & 1) + e])
+                         : "memory");
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_2d(&a.tdq, buf, 32 * quad, grow + 32 * c);
+            bulk_commit();
+          }
+        };
+        {
+          uint32_t v[64];
+          tmem_ld64(tDQ, v);
+          if (active) {
+            stage_chunk(v, 0);
+            stage_chunk(v, 1);
+          }
+        }
+        {
+          uint32_t v[64];
+          tmem_ld64(tDQ + 64, v);
+          tc_fence_before();
+          mbar_arrive(dq_free);
+          if (active) {
+            stage_chunk(v, 2);
+            stage_chunk(v, 3);
           }
         }
         (void)base;
