@@ -153,7 +153,8 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
 }
 
 // 2-D fp32 map over the dQ accumulator [H*rows][D] (row pitch D*4 bytes),
-// 32 x 32 boxes, no swizzle: the backward adds staged dQ tiles through it.
+// 32 x 32 boxes with 128-byte swizzle: the backward adds staged dQ tiles
+// through it.
 cudaError_t make_dq_map(CUtensorMap* map, float* base, int D, int64_t rows_total) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -162,7 +163,7 @@ cudaError_t make_dq_map(CUtensorMap* map, float* base, int D, int64_t rows_total
   cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

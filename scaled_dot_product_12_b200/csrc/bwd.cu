@@ -107,11 +107,11 @@ struct BwdCfg {
   static constexpr int kBlocks = DPAD / 64;
   static constexpr int kTileBytes = 128 * DPAD * 2;
   static constexpr int kQStages = 2;
-  // dQ^T path (head dim 128): the dQ tile is staged in shared memory for TMA
-  // bulk reductions (4 warps x 2 buffers x 32x32 fp32); dO gets one ring
-  // stage to make room.
-  static constexpr bool kStageDq = (DPAD == 128);
-  static constexpr int kDOStages = kStageDq ? 1 : 2;
+  // The dQ tile is staged in shared memory for TMA bulk reductions (4 warps x
+  // 2 buffers x 32x32 fp32); at head dim 128 dO gets one ring stage to make
+  // room.
+  static constexpr bool kStageDq = true;
+  static constexpr int kDOStages = (DPAD == 128) ? 1 : 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;
@@ -535,80 +535,84 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   } else {
     // ===================== dQ drain (warps 8-11) =====================
     const int quad = warp & 3;
-    const int t = quad * 32 + lane;  // TMEM lane of this thread
     const uint32_t tDQ = tmem + ((uint32_t)(quad * 32) << 16) + C::kColDQ;
+    const uint32_t stage = sDQ + quad * 8192;
+    int nbox = 0;  // boxes staged so far: alternates the two buffers across tiles
     for (int it = 0; it < n_it; ++it) {
       bool ok = mbar_wait(dq_mma, it & 1, abort_flag, a.status, kSiteDq);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int32_t m0 = (mb + it) * 128;
       const int64_t row0 = a.packed ? (int64_t)(qrow0 + m0) : (int64_t)b * a.Sq + m0;
-      float* base = a.dq_acc + ((int64_t)h * a.rows + row0) * a.D;
+      // Each warp stages 32 x 32 fp32 boxes (32 rows of the accumulator x 32
+      // head-dim columns, 128-byte swizzled like the tensor map) in one of its
+      // two buffers and adds them with a TMA bulk reduction.  Rows of queries
+      // outside the sequence hold exact zeros (their dS is 0), so whole boxes
+      // can be added; columns past D are clipped by the tensor map.
+      const int grow = (int)((int64_t)h * a.rows + row0);
+      auto issue_box = [&](uint32_t buf, int col, int row) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_2d(&a.tdq, buf, col, row);
+          bulk_commit();
+        }
+      };
+      auto next_buf = [&]() -> uint32_t {
+        const uint32_t buf = stage + (nbox & 1) * 4096;
+        ++nbox;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        return buf;
+      };
       if (C::kDqTransposed) {
-        // lane t = head-dim index d, column = query: a warp adds 32 consecutive
-        // floats of one query row per instruction.  The whole tile is pulled
-        // into registers first and the TMEM columns released before the
-        // reductions are issued, so the next MMA into them need not wait.
-        // Two 64-query halves: the first half is staged before the second is
-        // read, then the TMEM columns are released and the second staged.
-        // Each 32-query chunk becomes a 32 x 32 box (query rows x this warp's
-        // head-dim columns) added by a TMA bulk reduction; rows of queries
-        // outside the sequence hold exact zeros (their dS is 0).
+        // lane = head-dim index d (this warp: columns 32 quad .. +31), TMEM
+        // column = query.  Box rows are queries; each lane writes one float
+        // per row.  Read in two 64-query halves; TMEM is released after the
+        // second half is in registers.
         const bool active = 32 * quad < a.D;
-        const uint32_t stage = sDQ + quad * 8192;
-        const int grow = (int)((int64_t)h * a.rows + row0);
-        auto stage_chunk = [&](const uint32_t (&v)[64], int c) {
-          const uint32_t buf = stage + (c & 1) * 4096;
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + e * 128 + lane * 4),
-                         "r"(v[32 * (c & 1) + e])
-                         : "memory");
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_reduce_add_2d(&a.tdq, buf, 32 * quad, grow + 32 * c);
-            bulk_commit();
-          }
-        };
-        {
+        for (int hq = 0; hq < 2; ++hq) {
           uint32_t v[64];
-          tmem_ld64(tDQ, v);
+          tmem_ld64(tDQ + 64 * hq, v);
+          if (hq == 1) {
+            tc_fence_before();
+            mbar_arrive(dq_free);
+          }
           if (active) {
-            stage_chunk(v, 0);
-            stage_chunk(v, 1);
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const uint32_t buf = next_buf();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const uint32_t off = e * 128 + ((((uint32_t)lane >> 2) ^ (e & 7)) << 4) + (lane & 3) * 4;
+                asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + off), "r"(v[32 * c2 + e]) : "memory");
+              }
+              issue_box(buf, 32 * quad, grow + 64 * hq + 32 * c2);
+            }
           }
         }
-        {
-          uint32_t v[64];
-          tmem_ld64(tDQ + 64, v);
-          tc_fence_before();
-          mbar_arrive(dq_free);
-          if (active) {
-            stage_chunk(v, 2);
-            stage_chunk(v, 3);
-          }
-        }
-        (void)base;
-        continue;
       } else {
-        const bool valid = m0 + t < sq;
-        float* dst = base + (int64_t)t * a.D;
-        for (int c = 0; c < a.D / 16; ++c) {
-          uint32_t v[16];
-          tmem_ld16(tDQ + 16 * c, v);
-          if (valid) {
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              red_add_v4(dst + 16 * c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                         __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        // lane = query row (this warp: rows 32 quad .. +31), TMEM column =
+        // head-dim index.  Each lane writes its row's 32 floats of a box.
+        for (int cc = 0; cc < (a.D + 31) / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tDQ + 32 * cc, v);
+          if (32 * cc + 32 >= a.D) {  // last chunk read: TMEM can be reused
+            tc_fence_before();
+            mbar_arrive(dq_free);
           }
+          const uint32_t buf = next_buf();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = lane * 128 + (((uint32_t)k ^ (lane & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off), "r"(v[4 * k]),
+                         "r"(v[4 * k + 1]), "r"(v[4 * k + 2]), "r"(v[4 * k + 3])
+                         : "memory");
+          }
+          issue_box(buf, 32 * cc, grow + 32 * quad);
         }
       }
-      tc_fence_before();
-      mbar_arrive(dq_free);
     }
     // The staged tiles must stay in place until the TMA has added them.
     if (C::kStageDq && lane == 0) bulk_wait<0>();
