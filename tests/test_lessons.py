@@ -185,3 +185,21 @@ def test_bottom_right_fully_masked_rows(packed):
         assert np.all(o[..., empty[0, 0], :] == 0) and np.all(dq[..., empty[0, 0], :] == 0)
     assert_grads([got[n].float().numpy() for n in ("dq", "dk", "dv")],
                  [want[n] for n in ("dq", "dk", "dv")])
+
+
+@pytest.mark.parametrize("shape", [(512, 16, 384, 64), (4, 16, 384, 128), (2, 8, 2000, 128)])
+def test_repeated_runs_never_time_out(shape):
+    # Each query tile's softmax warps can run a step ahead of the MMA thread;
+    # a barrier reused across steps once let a fast group lap its consumer and
+    # stall it until the bounded wait gave up.  Repeat the shapes where that
+    # showed up and require a clean device status after every run.
+    B = binding()
+    dev = torch.device("cuda")
+    Bb, H, S, D = shape
+    q, k, v, do = (t.to(dev) for t in dense_inputs(Bb, H, S, S, D, torch.bfloat16, 91))
+    o, lse = B.forward(q, k, v)
+    for _ in range(10):
+        B.forward(q, k, v, out=o, lse=lse)
+        B.backward(do, q, k, v, o, lse)
+        torch.cuda.synchronize()
+        assert B.device_status(dev) == 0
