@@ -321,7 +321,11 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     a.total_q = p->total_q;
     a.rows = rows_q;
     a.sm_scale = p->sm_scale;
+    // c = sm_scale * log2(e); the kernel subtracts LSE*log2(e)/c inside the
+    // S^T product, so |c| is kept at least 2^-100.  Below that c * S^T is far
+    // under the rounding of LSE*log2(e) and P is unchanged in fp32.
     a.scale_log2 = p->sm_scale * 1.4426950408889634f;
+    if (std::fabs(a.scale_log2) < 0x1p-100f) a.scale_log2 = std::signbit(a.scale_log2) ? -0x1p-100f : 0x1p-100f;
     const size_t delta_bytes = ((size_t)p->H * rows_q * 4 + 255) & ~(size_t)255;
     a.delta = static_cast<float*>(p->workspace);
     a.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(p->workspace) + delta_bytes);

@@ -99,31 +99,45 @@ __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_const
 template <int DPAD>
 struct BwdCfg {
   // Warps 0-7: two P/dS groups (query columns 0-63 and 64-127 of every key
-  // row); 8-11: dQ drain; 12: TMA; 13: MMA.  14 warps: at most 4 per
-  // sub-partition, so 128 registers per thread.
-  static constexpr int kThreads = 448;
+  // row); 8-11: dQ drain; 12: TMA; 13: MMA; 14-15 idle.  16 warps, four per
+  // sub-partition, launch with 128 registers per thread; the TMA/MMA
+  // warpgroup then gives registers to the P/dS and drain warpgroups
+  // (setmaxnreg), so the drain can hold a whole 128-column dQ tile and
+  // release its TMEM columns right after reading them.
+  static constexpr int kThreads = 512;
+  static constexpr int kLaunchRegs = 128;
+  static constexpr int kProducerRegs = 96;
+  static constexpr int kDrainRegs = 144;
+  static constexpr int kPdsRegs = 136;
   static constexpr int kLoadWarp = 12;
   static constexpr int kMmaWarp = 13;
   static constexpr int kBlocks = DPAD / 64;
   static constexpr int kTileBytes = 128 * DPAD * 2;
   static constexpr int kQStages = 2;
   // The dQ tile is staged in shared memory for TMA bulk reductions (4 warps x
-  // 2 buffers x 32x32 fp32); at head dim 128 dO gets one ring stage to make
-  // room.
+  // kDqBufs buffers x 32x32 fp32); at head dim 128 dO gets one ring stage and
+  // each drain warp one staging buffer, to make room.
   static constexpr bool kStageDq = true;
   static constexpr int kDOStages = (DPAD == 128) ? 1 : 2;
+  static constexpr int kDqBufs = (DPAD == 128) ? 1 : 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;
   static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
   static constexpr int kOffDS = kOffDO + kDOStages * kTileBytes;  // 128 x 128 16-bit
   static constexpr int kOffDQ = kOffDS + 128 * 128 * 2;
-  static constexpr int kDqStageBytes = kStageDq ? 4 * 2 * 32 * 32 * 4 : 0;
-  static constexpr int kOffRow = kOffDQ + kDqStageBytes;           // lse/delta [2][2][128] f32
-  static constexpr int kOffBar = kOffRow + 2 * 2 * 128 * 4;
+  static constexpr int kDqStageBytes = kStageDq ? 4 * kDqBufs * 32 * 32 * 4 : 0;
+  // Operands of one extra 16-wide K step appended to the S^T and dP^T
+  // products, which subtracts the per-query constants inside the MMA (no-
+  // swizzle K-major, 128 rows x 16 bf16 = 4 KiB each): [0] ones on the key
+  // side, [1] -LSE/c terms of the next S^T tile, [2] -delta terms of the next
+  // dP^T tile, on the query side.
+  static constexpr int kXBytes = 128 * 16 * 2;
+  static constexpr int kOffX = kOffDQ + kDqStageBytes;
+  static constexpr int kOffBar = kOffX + 3 * kXBytes;
   // kv_full, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
-  // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 7;
+  // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done, x_ready
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 8;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + DPAD;
@@ -173,7 +187,7 @@ __device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t
 }
 
 template <int DPAD, bool BF16>
-__global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<DPAD>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -222,7 +236,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
 
   const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV, sQ = sbase + C::kOffQ,
                  sDO = sbase + C::kOffDO, sDS = sbase + C::kOffDS, sDQ = sbase + C::kOffDQ;
-  float* row_s = reinterpret_cast<float*>(smem + C::kOffRow);  // [buf][lse|delta][128]
+  const uint32_t sXA = sbase + C::kOffX, sXQ = sXA + C::kXBytes, sXD = sXA + 2 * C::kXBytes;
   const uint32_t bar0 = sbase + C::kOffBar;
   const uint32_t kv_full = bar0;
   auto q_full = [&](int s) { return bar0 + 8 * (1 + s); };
@@ -231,7 +245,8 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   auto do_empty = [&](int s) { return bar0 + 8 * (1 + 2 * C::kQStages + C::kDOStages + s); };
   const uint32_t s_full = bar0 + 8 * (1 + 2 * C::kQStages + 2 * C::kDOStages);
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24,
-                 dq_mma = s_full + 32, dq_free = s_full + 40, acc_done = s_full + 48;
+                 dq_mma = s_full + 32, dq_free = s_full + 40, acc_done = s_full + 48,
+                 x_ready = s_full + 56;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -252,6 +267,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(dq_mma, 1);
     mbar_init(dq_free, 128);
     mbar_init(acc_done, 1);
+    mbar_init(x_ready, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -265,6 +281,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 12) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kProducerRegs));
   if (warp == C::kLoadWarp) {
     // ===================== TMA producer =====================
     if (lane == 0) {
@@ -332,17 +349,25 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       const uint32_t loDOm = (uint32_t)make_sdesc(sDO, 16384, 1024);
       const uint32_t loDSm = (uint32_t)make_sdesc(sDS, 16384, 1024);
       constexpr uint32_t kTile16 = C::kTileBytes >> 4;
+      // The extra K step: always bf16 operands (a separate instruction, so
+      // independent of the inputs' type), accumulating into the same tile.
+      const uint32_t idesc_x = make_idesc(true, 128, 128, false, false);
+      const uint64_t dXA = make_sdesc_plain(sXA, 128, 256), dXQ = make_sdesc_plain(sXQ, 128, 256),
+                     dXD = make_sdesc_plain(sXD, 128, 256);
       bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma) &&
-                mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma);
+                mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma) &&
+                mbar_wait(x_ready, 0, abort_flag, a.status, kSiteMma);
       if (ok) {
         tc_fence_after();
         bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ, hiK, idesc_kk);
+        mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
         tc_commit(s_full);
         ok = mbar_wait(do_full(0), 0, abort_flag, a.status, kSiteMma);
       }
       if (ok) {
         tc_fence_after();
         bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO, hiK, idesc_kk);
+        mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
         tc_commit(dp_full);
       }
       for (int it = 0; it < n_it && ok; ++it) {
@@ -359,6 +384,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
           if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
           tc_fence_after();
           bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ + nqs * kTile16, hiK, idesc_kk);
+          mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
           tc_commit(s_full);
         }
         // dK += dS^T Q
@@ -382,6 +408,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
             break;
           tc_fence_after();
           bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + ndos * kTile16, hiK, idesc_kk);
+          mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
           tc_commit(dp_full);
         }
       }
@@ -389,6 +416,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     }
   }
   } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kPdsRegs));
     // ===================== P, dS and the dK / dV epilogue =====================
     // Group `half` owns query columns [64 half, 64 half + 64) of every key row.
     const int half = warp >> 2, quad = warp & 3;
@@ -398,14 +426,14 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
     const int qo = 64 * half;          // first query column of this group
     const uint32_t po = 64 * half;     // its P / dS columns (16-bit pairs)
-    const float sl2 = a.scale_log2;
+    const float sl2 = a.scale_log2;  // c = sm_scale * log2(e), |c| >= 2^-100
     // Queries that see key j: j - R <= i <= j + L, 0 <= i < sq (none if j >= sk).
     int32_t qa = j - win.R, qz = j + win.L;
     if (qa < 0) qa = 0;
     if (qz > sq - 1) qz = sq - 1;
     if (j >= sk) qz = qa - 1;
-    // Per-query values of a tile, one per thread: group 0 fetches LSE*log2(e),
-    // group 1 fetches delta, for query row r.
+    // Per-query values of a tile, one per thread: group 0 fetches LSE, group
+    // 1 fetches delta, for query row r (0 past the sequence).
     auto row_val = [&](int it) -> float {
       const int32_t i = (mb + it) * 128 + r;
       if (i >= sq) return 0.f;
@@ -415,29 +443,58 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
           li = a.lse_th ? (int64_t)(qrow0 + i) * a.H + h : (int64_t)h * a.total_q + qrow0 + i;
         else
           li = a.lse_th ? ((int64_t)b * a.Sq + i) * a.H + h : ((int64_t)b * a.H + h) * a.Sq + i;
-        return a.lse[li] * 1.4426950408889634f;
+        return a.lse[li];
       }
       const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
       return a.delta[(int64_t)h * a.rows + row];
     };
-    float val_n = row_val(0);
+    // The per-query constants enter the products through the extra K step:
+    // thread r writes query r's row of the query-side operand, the value as
+    // three bf16 terms (hi + mid + lo equals the fp32 value) in columns 0-2
+    // against ones in columns 0-2 of the key-side operand; columns 3-15 are 0.
+    // Group 0 writes -LSE*log2(e)/c (S^T*c - LSE*log2(e) == c*(S^T - that)),
+    // group 1 writes -delta.  Rows whose LSE is not finite (no allowed key)
+    // get 0: their P is zero through the column mask.
+    const uint32_t xrow = (uint32_t)((r >> 3) * 256 + (r & 7) * 16);  // core matrix (r/8, 0)
+    const float inv_c = 1.f / sl2;
+    auto folded = [&](float v) -> float {
+      if (half == 1) return -v;
+      return (v == -INFINITY || v == INFINITY || v != v) ? 0.f : -(v * 1.4426950408889634f) * inv_c;
+    };
+    auto put_row = [&](uint32_t base, float x) {
+      const uint32_t w_hi = pack2<true>(x, 0.f);
+      const float t0 = __uint_as_float(w_hi << 16);
+      const float r1 = x - t0;
+      const uint32_t w_mid = pack2<true>(r1, 0.f);
+      const float t1 = __uint_as_float(w_mid << 16);
+      const uint32_t w_lo = pack2<true>(r1 - t1, 0.f);
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(base + xrow),
+                   "r"((w_hi & 0xFFFFu) | (w_mid << 16)), "r"(w_lo & 0xFFFFu)
+                   : "memory");
+    };
+    {
+      // Constant parts, then tile 0's terms; the MMA issuer waits on x_ready.
+      const uint32_t one2 = pack2<true>(1.f, 1.f), one_ = pack2<true>(1.f, 0.f);
+      if (half == 0) {
+        st_shared_v4(sXA + xrow, one2, one_, 0u, 0u);
+        st_shared_v4(sXA + xrow + 128, 0u, 0u, 0u, 0u);
+      }
+      const uint32_t xb = half == 0 ? sXQ : sXD;
+      st_shared_v4(xb + xrow, 0u, 0u, 0u, 0u);
+      st_shared_v4(xb + xrow + 128, 0u, 0u, 0u, 0u);
+      put_row(xb, folded(row_val(0)));
+      fence_proxy_async_smem();
+      mbar_arrive(x_ready);
+    }
+    float v_next = n_it > 1 ? row_val(1) : 0.f;  // this group's value for tile it + 1
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int buf = it & 1;
-      float* lse_s = row_s + buf * 256;
-      float* dl_s = lse_s + 128;
-      (half == 0 ? lse_s : dl_s)[r] = val_n;
-      // Every warp of both groups passes this barrier once per tile, aborted
-      // or not, so none can be left waiting at it.
-      named_bar_sync(1, 256);
-      if (!ok) continue;
-      if (it + 1 < n_it) val_n = row_val(it + 1);
+    for (int it = 0; it < n_it && ok; ++it) {
       const int32_t m0 = (mb + it) * 128;
       const bool full = tile_is_full(win, sq, sk, m0, n0);
       const int32_t ca = qa - m0, cz = qz - m0;  // allowed columns [ca, cz]
-      // ---- phase 1: P^T = exp2(S^T * c*log2(e) - LSE*log2(e)), masked ----
+      // ---- phase 1: P^T = exp2(c * (S^T - LSE*log2(e)/c)), masked ----
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax));
-      if (!ok) continue;
+      if (!ok) break;
       tc_fence_after();
       // P is kept as the rounded 16-bit pairs the dV product uses.
       uint32_t pk[32];
@@ -445,18 +502,12 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       for (int c = 0; c < 2; ++c) {
         uint32_t sr[32];
         tmem_ld32(tS + qo + 32 * c, sr);
-        float lv[32];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const float4 t4 = reinterpret_cast<const float4*>(lse_s)[(qo >> 2) + 8 * c + jj];
-          lv[4 * jj] = t4.x; lv[4 * jj + 1] = t4.y; lv[4 * jj + 2] = t4.z; lv[4 * jj + 3] = t4.w;
-        }
         uint32_t chunk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int q0 = qo + 32 * c + 2 * e, q1 = q0 + 1;
-          float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, -lv[2 * e]));
-          float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -lv[2 * e + 1]));
+          float v0 = ex2(__uint_as_float(sr[2 * e]) * sl2);
+          float v1 = ex2(__uint_as_float(sr[2 * e + 1]) * sl2);
           if (!full) {
             v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
             v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
@@ -466,31 +517,31 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         }
         tmem_st16(tS + po + 16 * c, chunk);
       }
+      if (half == 0) {
+        // S^T(it) has been read: the operand can take tile it+1's terms.
+        if (it + 1 < n_it) put_row(sXQ, folded(v_next));
+        if (it + 2 < n_it) v_next = row_val(it + 2);
+      }
       tmem_wait_st();
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_ready);
       // ---- phase 2: dS^T = P^T o (dP^T - delta), into TMEM and shared memory ----
       ok = mbar_wait(dp_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
            (it == 0 || mbar_wait(dq_mma, (it - 1) & 1, abort_flag, a.status, kSiteSoftmax));
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) continue;
+      if (!ok) break;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
-        tmem_ld32(tDP + qo + 32 * c, dr);  // 32 queries of dP^T
-        float dv[32];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const float4 t4 = reinterpret_cast<const float4*>(dl_s)[(qo >> 2) + 8 * c + jj];
-          dv[4 * jj] = t4.x; dv[4 * jj + 1] = t4.y; dv[4 * jj + 2] = t4.z; dv[4 * jj + 3] = t4.w;
-        }
+        tmem_ld32(tDP + qo + 32 * c, dr);  // 32 queries of dP^T - delta
         uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 pe = unpack2<BF16>(pk[16 * c + e]);
-          const float d0 = pe.x * (__uint_as_float(dr[2 * e]) - dv[2 * e]);
-          const float d1 = pe.y * (__uint_as_float(dr[2 * e + 1]) - dv[2 * e + 1]);
+          const float d0 = pe.x * __uint_as_float(dr[2 * e]);
+          const float d1 = pe.y * __uint_as_float(dr[2 * e + 1]);
           dd[e] = pack2<BF16>(d0, d1);
         }
         tmem_st16(tDP + po + 16 * c, dd);
@@ -504,6 +555,11 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
                        "r"(dd[4 * u]), "r"(dd[4 * u + 1]), "r"(dd[4 * u + 2]), "r"(dd[4 * u + 3])
                        : "memory");
         }
+      }
+      if (half == 1) {
+        // dP^T(it) (delta subtracted in the MMA) has been read: next tile's terms.
+        if (it + 1 < n_it) put_row(sXD, folded(v_next));
+        if (it + 2 < n_it) v_next = row_val(it + 2);
       }
       fence_proxy_async_smem();
       tmem_wait_st();
@@ -534,10 +590,11 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     }
   } else {
     // ===================== dQ drain (warps 8-11) =====================
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kDrainRegs));
     const int quad = warp & 3;
     const uint32_t tDQ = tmem + ((uint32_t)(quad * 32) << 16) + C::kColDQ;
-    const uint32_t stage = sDQ + quad * 8192;
-    int nbox = 0;  // boxes staged so far: alternates the two buffers across tiles
+    const uint32_t stage = sDQ + quad * (C::kDqBufs * 4096);
+    int nbox = 0;  // boxes staged so far: cycles through the kDqBufs buffers across tiles
     for (int it = 0; it < n_it; ++it) {
       bool ok = mbar_wait(dq_mma, it & 1, abort_flag, a.status, kSiteDq);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -559,37 +616,34 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         }
       };
       auto next_buf = [&]() -> uint32_t {
-        const uint32_t buf = stage + (nbox & 1) * 4096;
+        const uint32_t buf = stage + (nbox % C::kDqBufs) * 4096;
         ++nbox;
-        if (lane == 0) bulk_wait_read<1>();
+        if (lane == 0) bulk_wait_read<C::kDqBufs - 1>();
         __syncwarp();
         return buf;
       };
       if (C::kDqTransposed) {
         // lane = head-dim index d (this warp: columns 32 quad .. +31), TMEM
         // column = query.  Box rows are queries; each lane writes one float
-        // per row.  Read in two 64-query halves; TMEM is released after the
-        // second half is in registers.
+        // per row.  The whole tile is read into registers first, so its TMEM
+        // columns (shared with dP^T) are released before any staging.
         const bool active = 32 * quad < a.D;
+        uint32_t v0[64], v1[64];
+        tmem_ld64(tDQ, v0);
+        tmem_ld64(tDQ + 64, v1);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        if (active) {
 #pragma unroll
-        for (int hq = 0; hq < 2; ++hq) {
-          uint32_t v[64];
-          tmem_ld64(tDQ + 64 * hq, v);
-          if (hq == 1) {
-            tc_fence_before();
-            mbar_arrive(dq_free);
-          }
-          if (active) {
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint32_t buf = next_buf();
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-              const uint32_t buf = next_buf();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const uint32_t off = e * 128 + ((((uint32_t)lane >> 2) ^ (e & 7)) << 4) + (lane & 3) * 4;
-                asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + off), "r"(v[32 * c2 + e]) : "memory");
-              }
-              issue_box(buf, 32 * quad, grow + 64 * hq + 32 * c2);
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t off = e * 128 + ((((uint32_t)lane >> 2) ^ (e & 7)) << 4) + (lane & 3) * 4;
+              const uint32_t val = c4 < 2 ? v0[32 * c4 + e] : v1[32 * (c4 - 2) + e];
+              asm volatile("st.shared.b32 [%0], %1;" ::"r"(buf + off), "r"(val) : "memory");
             }
+            issue_box(buf, 32 * quad, grow + 32 * c4);
           }
         }
       } else {
@@ -631,9 +685,18 @@ template <int DPAD, bool BF16>
 static cudaError_t launch_main(const BwdArgs& a, cudaStream_t stream) {
   using C = BwdCfg<DPAD>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  // One warp of each warpgroup per sub-partition: P/dS, P/dS, drain, TMA/MMA.
+  static_assert(2 * C::kPdsRegs + C::kDrainRegs + C::kProducerRegs <= 4 * C::kLaunchRegs,
+                "register split exceeds the launch budget");
   auto kern = attn_bwd_kernel<DPAD, BF16>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  // The setmaxnreg.inc of the P/dS and drain warpgroups draws on what the
+  // TMA/MMA warpgroup gives back from kLaunchRegs; with fewer registers at
+  // launch it would wait forever, so refuse to launch instead.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < C::kLaunchRegs) return cudaErrorLaunchOutOfResources;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((a.Sk + 127) / 128, a.H, a.B);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(a);

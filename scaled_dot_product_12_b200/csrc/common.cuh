@@ -236,6 +236,19 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle, K-major: the operand is
+// made of 8-row x 16-byte core matrices (128 contiguous bytes each); LBO is
+// the byte stride between core matrices adjacent in K, SBO between those
+// adjacent in M/N (8 rows further).
+__device__ __forceinline__ uint64_t make_sdesc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version of sm_100; layout type 0 = no swizzle
+  return d;
+}
+
 // TMEM loads: 32 lanes x 32 bits, one row (lane) per thread, N consecutive
 // columns.  The wait is inside the same asm statement so no use of the
 // result can be scheduled before the data has arrived.
@@ -334,6 +347,11 @@ __device__ __forceinline__ float2 unpack2(uint32_t v) {
   }
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
