@@ -335,14 +335,20 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c < a || c > z) s[c] = -INFINITY;
       }
-      // Row maximum over 8 independent chains (short dependency chains).
+      // Row maximum over 8 independent chains of three-input maxima: chain k
+      // takes columns k, k+8, ..., k+120 (0-23 to start, 24-119 in pairs,
+      // 120-127 last).
       float m8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = s[k];
+      for (int k = 0; k < 8; ++k) m8[k] = fmax3(s[k], s[8 + k], s[16 + k]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], s[c + k], s[c + 8 + k]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[120 + k]);
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                             fmaxf(m8[6], m8[7]));
       const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2;
       // Lazy rescale: keep the running reference unless the new maximum
       // exceeds it by more than 2^8 (P stays below 256, exact in fp32 sums).
@@ -352,24 +358,31 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         m_used = m_tile;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // Scale-and-shift and the row sum run on packed fp32 pairs.
+      uint64_t l4[4] = {0, 0, 0, 0};
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t packed[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float x0 = s[32 * c + 2 * e], x1 = s[32 * c + 2 * e + 1];
-          float p0 = ex2(fmaf(x0, sl2, neg_m)), p1 = ex2(fmaf(x1, sl2, neg_m));
+          float y0, y1;
+          f2_unpack(f2_fma(f2_pack(x0, x1), sl2x2, negm2), y0, y1);
+          float p0 = ex2(y0), p1 = ex2(y1);
           if (!full) {
             p0 = (x0 == -INFINITY) ? 0.f : p0;
             p1 = (x1 == -INFINITY) ? 0.f : p1;
           }
-          l8[e & 7] += p0 + p1;
+          l4[e & 3] = f2_add(l4[e & 3], f2_pack(p0, p1));
           packed[e] = pack2<BF16>(p0, p1);
         }
         tmem_st16(tS + 16 * c, packed);
       }
-      const float rowsum = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      float la, lb, lc, ld;
+      f2_unpack(f2_add(l4[0], l4[1]), la, lb);
+      f2_unpack(f2_add(l4[2], l4[3]), lc, ld);
+      const float rowsum = (la + lb) + (lc + ld);
       l = alpha * l + rowsum;
       if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O_t must hold PV of the previous tile before it is rescaled.
