@@ -298,6 +298,11 @@ def run_gpu(args, rank, world, local):
                      "frac_of_peak": round(bwd_tf / peak, 4),
                      "frac_of_burst": round(bwd_tf / burst, 4)},
         "bwd_other_ms": round(ms_step - fwd_ms - main_ms, 4),
+        # The delta preprocess and the dQ conversion are HBM-bound: their
+        # algorithmic bytes over the rest of the step (both kernels and the
+        # gaps between launches) give a lower bound on their bandwidth.
+        "bwd_other": other_bandwidth(w, world, ms_step - fwd_ms - main_ms,
+                                     peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])),
         "frac_of_peak": {"measured_burst": round(value / world / burst, 4),
                          "measured_sustained": round(value / world / sustained, 4),
                          "datasheet_dense": round(value / world / DATASHEET_DENSE_BF16_TFLOPS, 4)},
@@ -316,6 +321,17 @@ def run_gpu(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
+
+
+def other_bandwidth(w, world, ms, hbm_gbs):
+    """Preprocess reads O, dO (2 x 2D bytes per row and head) and writes delta
+    (4) and the zeroed fp32 dQ accumulator (4D); the conversion reads the
+    accumulator (4D) and writes dQ (2D): (14 D + 4) bytes per row and head."""
+    rows = w.B * w.Sq * w.H  # the bench workloads are dense
+    nbytes = rows * (14 * w.D + 4) * world
+    gbs = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
+    return {"ms": round(ms, 4), "bytes": nbytes, "gbs": round(gbs, 1) if gbs else None,
+            "peak_gbs": hbm_gbs, "frac": round(gbs / hbm_gbs, 4) if gbs else None}
 
 
 def power_capped(clocks):
@@ -404,21 +420,27 @@ def oracle_sample(w: synth.Workload, rows: int):
 
 
 def oracle_step(w, inputs):
+    """One oracle forward and backward; returns their wall times (s)."""
     from oracle import attn_ref as ref
     qn, kn, vn, don = inputs
     # rows of a prefix keep their own mask only when the window does not
     # depend on seqlen_q; the default workloads are unmasked or top-left.
+    t0 = time.perf_counter()
     ref.forward(qn, kn, vn, w.D ** -0.5, w.window_left, w.window_right, w.bottom_right)
+    t1 = time.perf_counter()
     ref.backward(qn, kn, vn, don, w.D ** -0.5, w.window_left, w.window_right, w.bottom_right)
+    return t1 - t0, time.perf_counter() - t1
 
 
 def cpu_baseline(w: synth.Workload, rows: int = 0):
     inputs, flops = oracle_sample(w, rows)
-    t = time.perf_counter()
-    oracle_step(w, inputs)
-    dt = time.perf_counter() - t
+    t_f, t_b = oracle_step(w, inputs)
+    dt = t_f + t_b
+    pair_flops = flops / (14 * w.D)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu_count": os.cpu_count(),
+            "fwd_tflops": round(4 * w.D * pair_flops / t_f / 1e12, 6),
+            "bwd_tflops": round(10 * w.D * pair_flops / t_b / 1e12, 6),
             "sample": f"fp64 NumPy oracle, forward + backward of head (0,0) "
                       f"({'all' if rows <= 0 else rows} query rows x {w.Sk} keys, "
                       f"{flops / 1e9:.1f} GFLOP at 14*D per pair), {dt:.1f} s on "
@@ -433,9 +455,12 @@ def run_reference(args, rank, world):
     for _ in range(args.warmup):
         oracle_step(w, inputs)
     t = time.perf_counter()
+    t_f = t_b = 0.0
     for _ in range(args.steps):
-        oracle_step(w, inputs)
+        f_s, b_s = oracle_step(w, inputs)
+        t_f, t_b = t_f + f_s, t_b + b_s
     dt = (time.perf_counter() - t) / args.steps
+    pair_flops = flops / (14 * w.D)
     value = flops / dt / 1e12
     sample = (f"each step: fp64 NumPy oracle forward + backward of head (0,0), first {rows} "
               f"query rows against all {w.Sk} keys ({flops / 1e9:.2f} GFLOP)")
@@ -445,7 +470,10 @@ def run_reference(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": describe(w),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _blas_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample, "cpu_count": os.cpu_count(),
+                             "fwd_tflops": round(4 * w.D * pair_flops * args.steps / t_f / 1e12, 6),
+                             "bwd_tflops": round(10 * w.D * pair_flops * args.steps / t_b / 1e12,
+                                                 6)},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
