@@ -102,13 +102,23 @@ extern "C" {
  * VarlenMode (one byte): bit 0 stacked (0 = BHSD, 1 = 1THD), bits 2:1 length
  * (0 uniform, 1 cumulative sums, 2 per-sequence array), bits 4:3 position
  * (0 uniform, 1 reuse the cumulative sums, 2 second array), bits 7:5
- * reserved.  Supported: both sides ATTN_VARLEN_MODE_DENSE, or both sides
- * ATTN_VARLEN_MODE_PACKED; any other mode returns ATTN_ERROR_INVALID_VALUE.
+ * reserved.  Supported, the same mode on both sides:
+ *   ATTN_VARLEN_MODE_DENSE   BHSD, every batch Sq queries and Sk keys;
+ *   ATTN_VARLEN_MODE_PACKED  1THD, cu_seqlens_q / _k hold B + 1 cumulative
+ *                            lengths (the positions reuse them);
+ *   ATTN_VARLEN_MODE_PADDED  BHSD sized [B, H, Sq, D] / [B, H, Sk, D], with
+ *                            per-batch lengths: cu_seqlens_q / _k then hold
+ *                            B lengths each (not cumulative; clamped to
+ *                            [0, Sq] / [0, Sk]); rows past a batch's lengths
+ *                            are padding: never written, and their contents
+ *                            (NaN included) do not reach any result.
+ * Any other mode returns ATTN_ERROR_INVALID_VALUE.
  */
 #define ATTN_VARLEN_MODE(stacked, length, position) \
   ((uint32_t)(stacked) | ((uint32_t)(length) << 1) | ((uint32_t)(position) << 3))
 #define ATTN_VARLEN_MODE_DENSE ATTN_VARLEN_MODE(0, 0, 0)
 #define ATTN_VARLEN_MODE_PACKED ATTN_VARLEN_MODE(1, 1, 1)
+#define ATTN_VARLEN_MODE_PADDED ATTN_VARLEN_MODE(0, 2, 0)
 #define ATTN_LSE_HT 0u
 #define ATTN_LSE_TH 1u
 #define ATTN_DIAGONAL_TOP_LEFT 0u
@@ -122,7 +132,9 @@ extern "C" {
  * packed -- B sequences, Sq / Sk the largest seqlen_q / seqlen_k (they size
  * the launch; a sequence longer than them is an error of the caller),
  * total_q / total_k the rows of the packed tensors, cu_seqlens_q / _k device
- * arrays of B + 1 int32 cumulative lengths starting at 0.
+ * arrays of B + 1 int32 cumulative lengths starting at 0; padded -- dense
+ * tensors of B batches with Sq / Sk rows, cu_seqlens_q / _k device arrays of
+ * B int32 lengths (seqlen_q / seqlen_k of each batch).
  */
 typedef struct attn_fwd_params {
   uint32_t struct_size; /* sizeof(attn_fwd_params) */
@@ -139,7 +151,7 @@ typedef struct attn_fwd_params {
   float sm_scale;           /* any finite value, zero and negative included */
   int32_t window_left, window_right;
   uint32_t varlen_bits;
-  const int32_t* cu_seqlens_q; /* packed only, device memory */
+  const int32_t* cu_seqlens_q; /* packed / padded only, device memory */
   const int32_t* cu_seqlens_k;
 } attn_fwd_params;
 

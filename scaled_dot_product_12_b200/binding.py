@@ -38,6 +38,7 @@ def varlen_mode(stacked: int, length: int, position: int) -> int:
 
 MODE_DENSE = varlen_mode(0, 0, 0)
 MODE_PACKED = varlen_mode(1, 1, 1)
+MODE_PADDED = varlen_mode(0, 2, 0)
 
 
 def varlen_bits(qmode: int, kmode: int, lse_layout: int, diagonal: int) -> int:
@@ -156,8 +157,11 @@ class Problem:
     """Sizes, window and layout of one call, shared by forward and backward."""
 
     def __init__(self, q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
-                 max_seqlen_q, max_seqlen_k, lse_layout):
+                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q=None, seqlens_k=None):
         self.packed = cu_seqlens_q is not None
+        self.padded = seqlens_q is not None
+        if self.padded and (self.packed or seqlens_k is None):
+            raise ValueError("padded inputs need seqlens_q and seqlens_k (and no cu_seqlens)")
         if self.packed:
             if cu_seqlens_k is None or max_seqlen_q is None or max_seqlen_k is None:
                 raise ValueError("packed inputs need cu_seqlens_q/_k and max_seqlen_q/_k")
@@ -177,10 +181,12 @@ class Problem:
         self.window = (int(window[0]), int(window[1]))
         self.bottom_right = bool(bottom_right)
         self.lse_th = (lse_layout.upper() == "TH")
-        mode = MODE_PACKED if self.packed else MODE_DENSE
+        mode = MODE_PACKED if self.packed else (MODE_PADDED if self.padded else MODE_DENSE)
         self.bits = varlen_bits(mode, mode, LSE_TH if self.lse_th else LSE_HT,
                                 DIAGONAL_BOTTOM_RIGHT if self.bottom_right else DIAGONAL_TOP_LEFT)
-        self.cu_q, self.cu_k = cu_seqlens_q, cu_seqlens_k
+        # padded: the pointer fields carry B per-batch lengths instead of sums
+        self.cu_q, self.cu_k = (seqlens_q, seqlens_k) if self.padded else (cu_seqlens_q,
+                                                                          cu_seqlens_k)
 
     def lse_shape(self):
         if self.packed:
@@ -202,15 +208,17 @@ class Problem:
 
 def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_right=False,
             cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None,
-            lse_layout="HT", out=None, lse=None, return_lse=True, stream=None
-            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            lse_layout="HT", out=None, lse=None, return_lse=True, stream=None,
+            seqlens_q=None, seqlens_k=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """O (and LSE) of FlashAttention through attn_fwd.
 
     Dense: q [B,H,Sq,D], k/v [B,H,Sk,D].  Packed: q [Tq,H,D], k/v [Tk,H,D] with
-    int32 cu_seqlens on the device and the largest sequence lengths.
+    int32 cu_seqlens on the device and the largest sequence lengths.  Padded:
+    dense shapes plus int32 seqlens_q / seqlens_k [B] on the device; rows past
+    a batch's lengths are left untouched.
     """
     pr = Problem(q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
-                 max_seqlen_q, max_seqlen_k, lse_layout)
+                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k)
     if out is None:
         out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
     if lse is None and return_lse:
@@ -247,10 +255,10 @@ def workspace_bytes(p: BwdParams) -> int:
 def backward(dout, q, k, v, o, lse, sm_scale=None, window=(WINDOW_INF, WINDOW_INF),
              bottom_right=False, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
              max_seqlen_k=None, lse_layout="HT", dq=None, dk=None, dv=None, workspace=None,
-             stream=None):
+             stream=None, seqlens_q=None, seqlens_k=None):
     """(dQ, dK, dV) through attn_bwd; the workspace is allocated if not given."""
     pr = Problem(q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
-                 max_seqlen_q, max_seqlen_k, lse_layout)
+                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

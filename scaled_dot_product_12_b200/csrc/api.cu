@@ -96,7 +96,8 @@ constexpr uint32_t kReservedBits = 0xFFF80000u;  // bits 31:19
 constexpr uint32_t kModeReserved = 0xE0u;        // bits 7:5 of a VarlenMode
 
 struct Mode {
-  bool packed;
+  bool packed;  // 1THD with cumulative lengths
+  bool padded;  // BHSD with per-batch lengths
   bool lse_th;
   bool bottom_right;
 };
@@ -106,9 +107,11 @@ bool decode_bits(uint32_t bits, Mode* m) {
   const uint32_t qm = bits & 0xFFu, km = (bits >> 8) & 0xFFu, lse = (bits >> 16) & 3u;
   if ((qm | km) & kModeReserved) return false;
   if (qm != km) return false;  // mixed Q/K addressing: not supported
-  if (qm != ATTN_VARLEN_MODE_DENSE && qm != ATTN_VARLEN_MODE_PACKED) return false;
+  if (qm != ATTN_VARLEN_MODE_DENSE && qm != ATTN_VARLEN_MODE_PACKED && qm != ATTN_VARLEN_MODE_PADDED)
+    return false;
   if (lse > 1) return false;
   m->packed = (qm == ATTN_VARLEN_MODE_PACKED);
+  m->padded = (qm == ATTN_VARLEN_MODE_PADDED);
   m->lse_th = (lse == ATTN_LSE_TH);
   m->bottom_right = ((bits >> 18) & 1u) != 0;
   return true;
@@ -183,6 +186,8 @@ bool common_ok(const P* p, size_t want_size, Mode* m, bool check_pointers = true
       return false;
     if (check_pointers && p->B > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_k)) return false;
   }
+  if (m->padded && check_pointers && p->B > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_k))
+    return false;
   return true;
 }
 
@@ -234,6 +239,7 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
     a.wr = p->window_right;
     a.bottom_right = m.bottom_right;
     a.packed = m.packed;
+    a.padded = m.padded;
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.negate = p->sm_scale < 0.f;
@@ -316,6 +322,7 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     a.wr = p->window_right;
     a.bottom_right = m.bottom_right;
     a.packed = m.packed;
+    a.padded = m.padded;
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.total_q = p->total_q;

@@ -83,6 +83,10 @@ __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_const
     const int c = (int)(x % chunks);
     const int h = (int)(g / a.rows);
     const int64_t row = g % a.rows;
+    if (a.padded) {  // rows past a batch's seqlen_q are padding: not written
+      const int32_t len = min(max(a.cu_q[row / a.Sq], 0), a.Sq);
+      if (row % a.Sq >= len) continue;
+    }
     const float4* src = reinterpret_cast<const float4*>(a.dq_acc + g * a.D + 8 * c);
     const float4 u = src[0], v = src[1];
     const float s = a.sm_scale;
@@ -204,6 +208,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     sq = a.cu_q[b + 1] - qrow0;
     sk = a.cu_k[b + 1] - krow0;
     bcoord = 0;
+  } else if (a.padded) {
+    sq = min(max(a.cu_q[b], 0), a.Sq);
+    sk = min(max(a.cu_k[b], 0), a.Sk);
   }
   const int32_t n0 = ntile * 128;
   if (n0 >= sk) return;
@@ -354,10 +361,22 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       const uint32_t idesc_x = make_idesc(true, 128, 128, false, false);
       const uint64_t dXA = make_sdesc_plain(sXA, 128, 256), dXQ = make_sdesc_plain(sXQ, 128, 256),
                      dXD = make_sdesc_plain(sXD, 128, 256);
+      // Padded batches: tile rows past seqlen_q / seqlen_k hold the caller's
+      // padding, not TMA zero fill; P and dS are 0 there, but 0 * NaN is not,
+      // so those rows are zeroed before the tensor cores first read a tile.
+      auto clear_padding = [&](uint32_t tile, int r0) {
+        if (a.padded && r0 < 128) {
+          zero_tile_rows(tile, r0, C::kBlocks);
+          fence_proxy_async_smem();
+        }
+      };
       bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma) &&
                 mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma) &&
                 mbar_wait(x_ready, 0, abort_flag, a.status, kSiteMma);
       if (ok) {
+        clear_padding(sK, sk - n0);
+        clear_padding(sV, sk - n0);
+        clear_padding(sQ, sq - mb * 128);
         tc_fence_after();
         bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ, hiK, idesc_kk);
         mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
@@ -365,6 +384,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         ok = mbar_wait(do_full(0), 0, abort_flag, a.status, kSiteMma);
       }
       if (ok) {
+        clear_padding(sDO, sq - mb * 128);
         tc_fence_after();
         bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO, hiK, idesc_kk);
         mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
@@ -382,6 +402,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         tc_commit(do_empty(dos));
         if (nx < n_it) {
           if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
+          clear_padding(sQ + nqs * C::kTileBytes, sq - (mb + nx) * 128);
           tc_fence_after();
           bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ + nqs * kTile16, hiK, idesc_kk);
           mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
@@ -406,6 +427,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           if (!(ok = mbar_wait(do_full(ndos), ndpar, abort_flag, a.status, kSiteMma))) break;
           if (C::kAliasDQ && !(ok = mbar_wait(dq_free, it & 1, abort_flag, a.status, kSiteMma)))
             break;
+          clear_padding(sDO + ndos * C::kTileBytes, sq - (mb + nx) * 128);
           tc_fence_after();
           bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + ndos * kTile16, hiK, idesc_kk);
           mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);

@@ -379,6 +379,16 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+// Zeroes rows [r0, 128) of a 128-row tile of 16-bit elements stored as
+// `blocks` 64-column blocks of 128-byte rows, 16 KiB apart (whole rows, so
+// the swizzle inside a row does not matter).  One thread; the caller fences
+// the async proxy before the tensor cores read the tile.
+__device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0, int blocks) {
+  for (int blk = 0; blk < blocks; ++blk)
+    for (int r = r0 < 0 ? 0 : r0; r < 128; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) st_shared_v4(tile + blk * 16384 + r * 128 + c * 16, 0u, 0u, 0u, 0u);
+}
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),

@@ -96,6 +96,9 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
     sq = args.cu_q[b + 1] - qrow0;
     sk = args.cu_k[b + 1] - krow0;
     bcoord = 0;
+  } else if (args.padded) {
+    sq = min(max(args.cu_q[b], 0), args.Sq);
+    sk = min(max(args.cu_k[b], 0), args.Sk);
   }
   const int32_t m0 = mblk * 128 * NQ;
   if (m0 >= sq) return;
@@ -249,6 +252,16 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         ok = mbar_wait(q_full(t), 0, abort_flag, args.status, kSiteMma);
       // O_t (+)= P_t V: P from TMEM (16 columns of 32 bits per 16 keys... 8
       // columns per K step of 16 keys), V MN-major, next 16 keys = +2048 bytes.
+      // Padded batches: rows of a V tile past seqlen_k hold the caller's
+      // padding, not TMA zero fill; P is 0 there, but 0 * NaN is not, so the
+      // rows are zeroed before the tensor cores read the tile.
+      auto clear_v_padding = [&](int it_v) {
+        const int r0 = sk - (nb + it_v) * 128;
+        if (args.padded && r0 < 128) {
+          zero_tile_rows(sV + (it_v % C::kVStages) * C::kTileBytes, r0, C::kBlocks);
+          fence_proxy_async_smem();
+        }
+      };
       auto issue_pv = [=](int t, int it_prev) {
         fwd_issue_pv(tmem + C::kColO + DPAD * t, tmem + 128 * t,
                      dV + (uint32_t)(it_prev % C::kVStages) * kTile16, kHiV, idesc_o, it_prev > 0);
@@ -274,6 +287,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
               if (!(ok = mbar_wait(v_full(vs), ((it - 1) / C::kVStages) & 1, abort_flag,
                                    args.status, kSiteMma)))
                 break;
+              clear_v_padding(it - 1);
             }
             tc_fence_after();
             issue_pv(t, it - 1);
@@ -293,6 +307,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
             if (!(ok = mbar_wait(v_full(vs), (last / C::kVStages) & 1, abort_flag, args.status,
                                  kSiteMma)))
               break;
+            clear_v_padding(last);
           }
           tc_fence_after();
           issue_pv(t, last);

@@ -19,6 +19,7 @@ struct FwdArgs {
   const int32_t* cu_k;
   int32_t B, H, Sq, Sk, D;
   int32_t wl, wr, bottom_right, packed, lse_th, bf16, negate;
+  int32_t padded;  // BHSD with per-batch lengths in cu_q / cu_k (B entries each)
   int64_t total_q;
   float scale_log2;  // |sm_scale| * log2(e)
   uint32_t* status;
@@ -38,6 +39,7 @@ struct BwdArgs {
   const int32_t* cu_k;
   int32_t B, H, Sq, Sk, D;
   int32_t wl, wr, bottom_right, packed, lse_th, bf16;
+  int32_t padded;  // BHSD with per-batch lengths in cu_q / cu_k (B entries each)
   int64_t total_q, rows;  // rows of the workspace: B*Sq (dense) or total_q
   float sm_scale;
   float scale_log2;       // sm_scale * log2(e) (sign kept)
