@@ -102,16 +102,18 @@ extern "C" {
  * VarlenMode (one byte): bit 0 stacked (0 = BHSD, 1 = 1THD), bits 2:1 length
  * (0 uniform, 1 cumulative sums, 2 per-sequence array), bits 4:3 position
  * (0 uniform, 1 reuse the cumulative sums, 2 second array), bits 7:5
- * reserved.  Supported, the same mode on both sides:
- *   ATTN_VARLEN_MODE_DENSE   BHSD, every batch Sq queries and Sk keys;
- *   ATTN_VARLEN_MODE_PACKED  1THD, cu_seqlens_q / _k hold B + 1 cumulative
- *                            lengths (the positions reuse them);
+ * reserved.  Each side takes one of three modes on its own (the Q side
+ * addresses Q, O, LSE, dO and dQ; the K side K, V, dK and dV):
+ *   ATTN_VARLEN_MODE_DENSE   BHSD, every batch Sq queries / Sk keys;
+ *   ATTN_VARLEN_MODE_PACKED  1THD, that side's cu_seqlens array holds B + 1
+ *                            cumulative lengths (the positions reuse them);
  *   ATTN_VARLEN_MODE_PADDED  BHSD sized [B, H, Sq, D] / [B, H, Sk, D], with
- *                            per-batch lengths: cu_seqlens_q / _k then hold
- *                            B lengths each (not cumulative; clamped to
+ *                            per-batch lengths: that side's cu_seqlens array
+ *                            holds B lengths (not cumulative; clamped to
  *                            [0, Sq] / [0, Sk]); rows past a batch's lengths
  *                            are padding: never written, and their contents
  *                            (NaN included) do not reach any result.
+ * A batch index b names the same sequence on both sides.
  * Any other mode returns ATTN_ERROR_INVALID_VALUE.
  */
 #define ATTN_VARLEN_MODE(stacked, length, position) \

@@ -158,38 +158,53 @@ class Problem:
 
     def __init__(self, q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
                  max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q=None, seqlens_k=None):
-        self.packed = cu_seqlens_q is not None
-        self.padded = seqlens_q is not None
-        if self.padded and (self.packed or seqlens_k is None):
-            raise ValueError("padded inputs need seqlens_q and seqlens_k (and no cu_seqlens)")
-        if self.packed:
-            if cu_seqlens_k is None or max_seqlen_q is None or max_seqlen_k is None:
-                raise ValueError("packed inputs need cu_seqlens_q/_k and max_seqlen_q/_k")
-            if q.dim() != 3 or k.dim() != 3:
-                raise ValueError("packed inputs are [tokens, H, D]")
-            self.B = cu_seqlens_q.numel() - 1
-            self.H, self.D = q.shape[1], q.shape[2]
-            self.Sq, self.Sk = int(max_seqlen_q), int(max_seqlen_k)
-            self.total_q, self.total_k = q.shape[0], k.shape[0]
-        else:
-            if q.dim() != 4 or k.dim() != 4:
-                raise ValueError("dense inputs are [B, H, S, D]")
-            self.B, self.H, self.Sq, self.D = q.shape
-            self.Sk = k.shape[2]
-            self.total_q = self.total_k = 0
+        # Each side on its own: packed (cu_seqlens, 3-D [T, H, D] tensors),
+        # padded (seqlens, 4-D [B, H, S, D] tensors) or dense (4-D).
+        if cu_seqlens_q is not None and seqlens_q is not None or \
+                cu_seqlens_k is not None and seqlens_k is not None:
+            raise ValueError("a side is packed (cu_seqlens) or padded (seqlens), not both")
+        self.q_packed, self.k_packed = cu_seqlens_q is not None, cu_seqlens_k is not None
+        self.q_padded, self.k_padded = seqlens_q is not None, seqlens_k is not None
+        for name, packed, t in (("q", self.q_packed, q), ("k", self.k_packed, k)):
+            if t.dim() != (3 if packed else 4):
+                raise ValueError(f"{name}: packed inputs are [tokens, H, D], others [B, H, S, D]")
+        sizes = set()
+        if self.q_packed:
+            sizes.add(cu_seqlens_q.numel() - 1)
+        elif self.q_padded:
+            sizes.add(seqlens_q.numel())
+        if self.k_packed:
+            sizes.add(cu_seqlens_k.numel() - 1)
+        elif self.k_padded:
+            sizes.add(seqlens_k.numel())
+        if not self.q_packed:
+            sizes.add(q.shape[0])
+        if not self.k_packed:
+            sizes.add(k.shape[0])
+        if len(sizes) != 1:
+            raise ValueError(f"inconsistent batch / sequence counts {sorted(sizes)}")
+        self.B = sizes.pop()
+        self.H, self.D = (q.shape[1], q.shape[2]) if self.q_packed else (q.shape[1], q.shape[3])
+        if (self.q_packed and max_seqlen_q is None) or (self.k_packed and max_seqlen_k is None):
+            raise ValueError("a packed side needs its max_seqlen")
+        self.Sq = int(max_seqlen_q) if self.q_packed else q.shape[2]
+        self.Sk = int(max_seqlen_k) if self.k_packed else k.shape[2]
+        self.total_q = q.shape[0] if self.q_packed else 0
+        self.total_k = k.shape[0] if self.k_packed else 0
         self.sm_scale = float(sm_scale) if sm_scale is not None else self.D ** -0.5
         self.window = (int(window[0]), int(window[1]))
         self.bottom_right = bool(bottom_right)
         self.lse_th = (lse_layout.upper() == "TH")
-        mode = MODE_PACKED if self.packed else (MODE_PADDED if self.padded else MODE_DENSE)
-        self.bits = varlen_bits(mode, mode, LSE_TH if self.lse_th else LSE_HT,
+        qmode = MODE_PACKED if self.q_packed else (MODE_PADDED if self.q_padded else MODE_DENSE)
+        kmode = MODE_PACKED if self.k_packed else (MODE_PADDED if self.k_padded else MODE_DENSE)
+        self.bits = varlen_bits(qmode, kmode, LSE_TH if self.lse_th else LSE_HT,
                                 DIAGONAL_BOTTOM_RIGHT if self.bottom_right else DIAGONAL_TOP_LEFT)
-        # padded: the pointer fields carry B per-batch lengths instead of sums
-        self.cu_q, self.cu_k = (seqlens_q, seqlens_k) if self.padded else (cu_seqlens_q,
-                                                                          cu_seqlens_k)
+        # the pointer fields carry whichever array each side's mode names
+        self.cu_q = cu_seqlens_q if self.q_packed else seqlens_q
+        self.cu_k = cu_seqlens_k if self.k_packed else seqlens_k
 
     def lse_shape(self):
-        if self.packed:
+        if self.q_packed:
             return (self.total_q, self.H) if self.lse_th else (self.H, self.total_q)
         return (self.B, self.Sq, self.H) if self.lse_th else (self.B, self.H, self.Sq)
 
@@ -226,10 +241,10 @@ def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_righ
     p = FwdParams()
     pr.fill(p, _dtype_code(q))
     p.q, p.k, p.v, p.o, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse)
-    p.q_stride = _strides(q, pr.packed)
-    p.k_stride = _strides(k, pr.packed)
-    p.v_stride = _strides(v, pr.packed)
-    p.o_stride = _strides(out, pr.packed)
+    p.q_stride = _strides(q, pr.q_packed)
+    p.k_stride = _strides(k, pr.k_packed)
+    p.v_stride = _strides(v, pr.k_packed)
+    p.o_stride = _strides(out, pr.q_packed)
     _check("attn_fwd", lib().attn_fwd(ctypes.byref(p), _stream_handle(q.device, stream)))
     return out, lse
 
@@ -241,7 +256,8 @@ def bwd_params(dout, q, k, v, o, lse, pr: Problem, dq, dk, dv, workspace=None) -
     p.dq, p.dk, p.dv = _ptr(dq), _ptr(dk), _ptr(dv)
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", dout), ("dq", dq), ("dk", dk),
                     ("dv", dv)):
-        setattr(p, name + "_stride", _strides(t, pr.packed))
+        setattr(p, name + "_stride", _strides(t, pr.k_packed if name in ("k", "v", "dk", "dv")
+                                              else pr.q_packed))
     if workspace is not None:
         p.workspace = workspace.data_ptr()
         p.workspace_bytes = workspace.numel() * workspace.element_size()

@@ -95,9 +95,10 @@ cudaError_t on_stream_device(cudaStream_t stream, F&& fn) {
 constexpr uint32_t kReservedBits = 0xFFF80000u;  // bits 31:19
 constexpr uint32_t kModeReserved = 0xE0u;        // bits 7:5 of a VarlenMode
 
+// Addressing of each side (Q: Q, O, LSE, dO, dQ; K: K, V, dK, dV).
 struct Mode {
-  bool packed;  // 1THD with cumulative lengths
-  bool padded;  // BHSD with per-batch lengths
+  bool q_packed, k_packed;  // 1THD with cumulative lengths
+  bool q_padded, k_padded;  // BHSD with per-batch lengths
   bool lse_th;
   bool bottom_right;
 };
@@ -106,12 +107,15 @@ bool decode_bits(uint32_t bits, Mode* m) {
   if (bits & kReservedBits) return false;
   const uint32_t qm = bits & 0xFFu, km = (bits >> 8) & 0xFFu, lse = (bits >> 16) & 3u;
   if ((qm | km) & kModeReserved) return false;
-  if (qm != km) return false;  // mixed Q/K addressing: not supported
-  if (qm != ATTN_VARLEN_MODE_DENSE && qm != ATTN_VARLEN_MODE_PACKED && qm != ATTN_VARLEN_MODE_PADDED)
-    return false;
+  auto known = [](uint32_t x) {
+    return x == ATTN_VARLEN_MODE_DENSE || x == ATTN_VARLEN_MODE_PACKED || x == ATTN_VARLEN_MODE_PADDED;
+  };
+  if (!known(qm) || !known(km)) return false;  // each side on its own: dense, packed or padded
   if (lse > 1) return false;
-  m->packed = (qm == ATTN_VARLEN_MODE_PACKED);
-  m->padded = (qm == ATTN_VARLEN_MODE_PADDED);
+  m->q_packed = (qm == ATTN_VARLEN_MODE_PACKED);
+  m->k_packed = (km == ATTN_VARLEN_MODE_PACKED);
+  m->q_padded = (qm == ATTN_VARLEN_MODE_PADDED);
+  m->k_padded = (km == ATTN_VARLEN_MODE_PADDED);
   m->lse_th = (lse == ATTN_LSE_TH);
   m->bottom_right = ((bits >> 18) & 1u) != 0;
   return true;
@@ -181,13 +185,13 @@ bool common_ok(const P* p, size_t want_size, Mode* m, bool check_pointers = true
   if (p->Sq >= attn::kBig || p->Sk >= attn::kBig) return false;
   if (!std::isfinite(p->sm_scale)) return false;
   if (!decode_bits(p->varlen_bits, m)) return false;
-  if (m->packed) {
-    if (p->total_q < 0 || p->total_k < 0 || p->total_q >= attn::kBig || p->total_k >= attn::kBig)
-      return false;
-    if (check_pointers && p->B > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_k)) return false;
+  if (m->q_packed && (p->total_q < 0 || p->total_q >= attn::kBig)) return false;
+  if (m->k_packed && (p->total_k < 0 || p->total_k >= attn::kBig)) return false;
+  // Packed and padded sides read their lengths from the device arrays.
+  if (check_pointers && p->B > 0) {
+    if ((m->q_packed || m->q_padded) && !p->cu_seqlens_q) return false;
+    if ((m->k_packed || m->k_padded) && !p->cu_seqlens_k) return false;
   }
-  if (m->padded && check_pointers && p->B > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_k))
-    return false;
   return true;
 }
 
@@ -200,19 +204,19 @@ extern "C" {
 int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
   Mode m;
   if (!common_ok(p, sizeof(attn_fwd_params), &m)) return cudaErrorInvalidValue;
-  const int64_t rows_q = m.packed ? p->total_q : (int64_t)p->B * p->Sq;
-  const int64_t rows_k = m.packed ? p->total_k : (int64_t)p->B * p->Sk;
+  const int64_t rows_q = m.q_packed ? p->total_q : (int64_t)p->B * p->Sq;
+  const int64_t rows_k = m.k_packed ? p->total_k : (int64_t)p->B * p->Sk;
   if (!has_work(p->B, p->H, rows_q)) return cudaSuccess;
   if (!p->q || !p->o) return cudaErrorInvalidValue;
   if (rows_k > 0 && (!p->k || !p->v)) return cudaErrorInvalidValue;
   if (!aligned16(p->q) || !aligned16(p->o) || (rows_k > 0 && (!aligned16(p->k) || !aligned16(p->v))))
     return cudaErrorInvalidValue;
   if (p->lse && (reinterpret_cast<uintptr_t>(p->lse) & 3u)) return cudaErrorInvalidValue;
-  const int64_t nq = m.packed ? p->total_q : p->Sq, nk = m.packed ? p->total_k : p->Sk;
-  if (!strides_ok(p->q_stride, m.packed, p->B, p->H, nq) ||
-      !strides_ok(p->o_stride, m.packed, p->B, p->H, nq) ||
-      !strides_ok(p->k_stride, m.packed, p->B, p->H, nk) ||
-      !strides_ok(p->v_stride, m.packed, p->B, p->H, nk))
+  const int64_t nq = m.q_packed ? p->total_q : p->Sq, nk = m.k_packed ? p->total_k : p->Sk;
+  if (!strides_ok(p->q_stride, m.q_packed, p->B, p->H, nq) ||
+      !strides_ok(p->o_stride, m.q_packed, p->B, p->H, nq) ||
+      !strides_ok(p->k_stride, m.k_packed, p->B, p->H, nk) ||
+      !strides_ok(p->v_stride, m.k_packed, p->B, p->H, nk))
     return cudaErrorInvalidValue;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
@@ -221,9 +225,9 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
     std::memset(&a, 0, sizeof(a));
     const void* kbase = rows_k > 0 ? p->k : p->q;
     const void* vbase = rows_k > 0 ? p->v : p->q;
-    cudaError_t e = make_map(&a.tq, p->q, p->D, nq, p->H, p->B, p->q_stride, m.packed);
-    if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.packed);
-    if (e == cudaSuccess) e = make_map(&a.tv, vbase, p->D, nk, p->H, p->B, p->v_stride, m.packed);
+    cudaError_t e = make_map(&a.tq, p->q, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
+    if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
+    if (e == cudaSuccess) e = make_map(&a.tv, vbase, p->D, nk, p->H, p->B, p->v_stride, m.k_packed);
     if (e != cudaSuccess) return e;
     a.o = p->o;
     a.lse = p->lse;
@@ -238,8 +242,10 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
     a.wl = p->window_left;
     a.wr = p->window_right;
     a.bottom_right = m.bottom_right;
-    a.packed = m.packed;
-    a.padded = m.padded;
+    a.q_packed = m.q_packed;
+    a.k_packed = m.k_packed;
+    a.q_padded = m.q_padded;
+    a.k_padded = m.k_padded;
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.negate = p->sm_scale < 0.f;
@@ -253,7 +259,7 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
 size_t attn_bwd_workspace_size(const attn_bwd_params* p) {
   Mode m;
   if (!common_ok(p, sizeof(attn_bwd_params), &m, /*check_pointers=*/false)) return 0;
-  const int64_t rows = m.packed ? p->total_q : (int64_t)p->B * p->Sq;
+  const int64_t rows = m.q_packed ? p->total_q : (int64_t)p->B * p->Sq;
   const int64_t n = (int64_t)p->H * rows;
   const size_t delta_bytes = ((size_t)n * 4 + 255) & ~(size_t)255;
   return delta_bytes + (size_t)n * p->D * 4;
@@ -262,8 +268,8 @@ size_t attn_bwd_workspace_size(const attn_bwd_params* p) {
 int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
   Mode m;
   if (!common_ok(p, sizeof(attn_bwd_params), &m)) return cudaErrorInvalidValue;
-  const int64_t rows_q = m.packed ? p->total_q : (int64_t)p->B * p->Sq;
-  const int64_t rows_k = m.packed ? p->total_k : (int64_t)p->B * p->Sk;
+  const int64_t rows_q = m.q_packed ? p->total_q : (int64_t)p->B * p->Sq;
+  const int64_t rows_k = m.k_packed ? p->total_k : (int64_t)p->B * p->Sk;
   if (!has_work(p->B, p->H, rows_q) && !(p->B > 0 && p->H > 0 && rows_k > 0)) return cudaSuccess;
   const void* need16[] = {p->q, p->o, p->dout, p->dq};
   for (const void* x : need16)
@@ -277,13 +283,13 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
   if (ws > 0 && (!p->workspace || p->workspace_bytes < ws ||
                  (reinterpret_cast<uintptr_t>(p->workspace) & 255u)))
     return cudaErrorInvalidValue;
-  const int64_t nq = m.packed ? p->total_q : p->Sq, nk = m.packed ? p->total_k : p->Sk;
+  const int64_t nq = m.q_packed ? p->total_q : p->Sq, nk = m.k_packed ? p->total_k : p->Sk;
   const int64_t* sq_list[] = {p->q_stride, p->o_stride, p->do_stride, p->dq_stride};
   for (const int64_t* st : sq_list)
-    if (!strides_ok(st, m.packed, p->B, p->H, nq)) return cudaErrorInvalidValue;
+    if (!strides_ok(st, m.q_packed, p->B, p->H, nq)) return cudaErrorInvalidValue;
   const int64_t* sk_list[] = {p->k_stride, p->v_stride, p->dk_stride, p->dv_stride};
   for (const int64_t* st : sk_list)
-    if (!strides_ok(st, m.packed, p->B, p->H, nk)) return cudaErrorInvalidValue;
+    if (!strides_ok(st, m.k_packed, p->B, p->H, nk)) return cudaErrorInvalidValue;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   return on_stream_device(stream, [&](const DeviceInfo& info) -> cudaError_t {
@@ -293,10 +299,11 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     const void* dobase = rows_q > 0 ? p->dout : p->k;
     const void* kbase = rows_k > 0 ? p->k : p->q;
     const void* vbase = rows_k > 0 ? p->v : p->q;
-    cudaError_t e = make_map(&a.tq, qbase, p->D, nq, p->H, p->B, p->q_stride, m.packed);
-    if (e == cudaSuccess) e = make_map(&a.tdo, dobase, p->D, nq, p->H, p->B, p->do_stride, m.packed);
-    if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.packed);
-    if (e == cudaSuccess) e = make_map(&a.tv, vbase, p->D, nk, p->H, p->B, p->v_stride, m.packed);
+    cudaError_t e = make_map(&a.tq, qbase, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
+    if (e == cudaSuccess)
+      e = make_map(&a.tdo, dobase, p->D, nq, p->H, p->B, p->do_stride, m.q_packed);
+    if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
+    if (e == cudaSuccess) e = make_map(&a.tv, vbase, p->D, nk, p->H, p->B, p->v_stride, m.k_packed);
     if (e != cudaSuccess) return e;
     a.o = p->o;
     a.dout = p->dout;
@@ -321,8 +328,10 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     a.wl = p->window_left;
     a.wr = p->window_right;
     a.bottom_right = m.bottom_right;
-    a.packed = m.packed;
-    a.padded = m.padded;
+    a.q_packed = m.q_packed;
+    a.k_packed = m.k_packed;
+    a.q_padded = m.q_padded;
+    a.k_padded = m.k_padded;
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.total_q = p->total_q;

@@ -49,10 +49,10 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant
     if (sub < chunks) {
       const uint4 ov = *reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(a.o) +
-          2 * (row_offset(a.o_stride, row, h, a.Sq, a.packed) + 8 * sub));
+          2 * (row_offset(a.o_stride, row, h, a.Sq, a.q_packed) + 8 * sub));
       const uint4 dv = *reinterpret_cast<const uint4*>(
           reinterpret_cast<const uint8_t*>(a.dout) +
-          2 * (row_offset(a.do_stride, row, h, a.Sq, a.packed) + 8 * sub));
+          2 * (row_offset(a.do_stride, row, h, a.Sq, a.q_packed) + 8 * sub));
       const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_const
     const int c = (int)(x % chunks);
     const int h = (int)(g / a.rows);
     const int64_t row = g % a.rows;
-    if (a.padded) {  // rows past a batch's seqlen_q are padding: not written
+    if (a.q_padded) {  // rows past a batch's seqlen_q are padding: not written
       const int32_t len = min(max(a.cu_q[row / a.Sq], 0), a.Sq);
       if (row % a.Sq >= len) continue;
     }
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_const
     const float4 u = src[0], v = src[1];
     const float s = a.sm_scale;
     uint8_t* dst = reinterpret_cast<uint8_t*>(a.dq) +
-                   2 * (row_offset(a.dq_stride, row, h, a.Sq, a.packed) + 8 * c);
+                   2 * (row_offset(a.dq_stride, row, h, a.Sq, a.q_packed) + 8 * c);
     st_global_v4(dst, pack2<BF16>(u.x * s, u.y * s), pack2<BF16>(u.z * s, u.w * s),
                  pack2<BF16>(v.x * s, v.y * s), pack2<BF16>(v.z * s, v.w * s));
   }
@@ -201,15 +201,20 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   const int ntile = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
-  int32_t sq = a.Sq, sk = a.Sk, qrow0 = 0, krow0 = 0, bcoord = b;
-  if (a.packed) {
+  // Q and K sides are addressed independently (see the forward kernel).
+  int32_t sq = a.Sq, sk = a.Sk, qrow0 = 0, krow0 = 0, bq = b, bk = b;
+  if (a.q_packed) {
     qrow0 = a.cu_q[b];
-    krow0 = a.cu_k[b];
     sq = a.cu_q[b + 1] - qrow0;
-    sk = a.cu_k[b + 1] - krow0;
-    bcoord = 0;
-  } else if (a.padded) {
+    bq = 0;
+  } else if (a.q_padded) {
     sq = min(max(a.cu_q[b], 0), a.Sq);
+  }
+  if (a.k_packed) {
+    krow0 = a.cu_k[b];
+    sk = a.cu_k[b + 1] - krow0;
+    bk = 0;
+  } else if (a.k_padded) {
     sk = min(max(a.cu_k[b], 0), a.Sk);
   }
   const int32_t n0 = ntile * 128;
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   const int n_it = me - mb;
 
   auto kv_row_ptr = [&](void* base, const int64_t* st, int32_t j) -> uint8_t* {
-    int64_t off = a.packed ? (int64_t)(krow0 + j) * st[2]
+    int64_t off = a.k_packed ? (int64_t)(krow0 + j) * st[2]
                            : (int64_t)b * st[0] + (int64_t)j * st[2];
     off += (int64_t)h * st[1];
     return reinterpret_cast<uint8_t*>(base) + 2 * off;
@@ -298,8 +303,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       prefetch_tmap(&a.tdo);
       mbar_expect_tx(kv_full, 2 * C::kTileBytes);
       for (int blk = 0; blk < C::kBlocks; ++blk) {
-        tma_load_4d(sK + blk * 16384, &a.tk, kv_full, 64 * blk, krow0 + n0, h, bcoord);
-        tma_load_4d(sV + blk * 16384, &a.tv, kv_full, 64 * blk, krow0 + n0, h, bcoord);
+        tma_load_4d(sK + blk * 16384, &a.tk, kv_full, 64 * blk, krow0 + n0, h, bk);
+        tma_load_4d(sV + blk * 16384, &a.tv, kv_full, 64 * blk, krow0 + n0, h, bk);
       }
       int nq = 0, ndo = 0;
       for (int it = 0; it < n_it; ++it) {
@@ -310,7 +315,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         mbar_expect_tx(q_full(qs), C::kTileBytes);
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sQ + qs * C::kTileBytes + blk * 16384, &a.tq, q_full(qs), 64 * blk, qrow, h,
-                      bcoord);
+                      bq);
         ++nq;
         const int ds = it % C::kDOStages, dround = it / C::kDOStages;
         if (dround > 0 &&
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         mbar_expect_tx(do_full(ds), C::kTileBytes);
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sDO + ds * C::kTileBytes + blk * 16384, &a.tdo, do_full(ds), 64 * blk, qrow,
-                      h, bcoord);
+                      h, bq);
         ++ndo;
       }
       if (*abort_flag) {
@@ -361,80 +366,93 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       const uint32_t idesc_x = make_idesc(true, 128, 128, false, false);
       const uint64_t dXA = make_sdesc_plain(sXA, 128, 256), dXQ = make_sdesc_plain(sXQ, 128, 256),
                      dXD = make_sdesc_plain(sXD, 128, 256);
-      // Padded batches: tile rows past seqlen_q / seqlen_k hold the caller's
-      // padding, not TMA zero fill; P and dS are 0 there, but 0 * NaN is not,
-      // so those rows are zeroed before the tensor cores first read a tile.
-      auto clear_padding = [&](uint32_t tile, int r0) {
-        if (a.padded && r0 < 128) {
-          zero_tile_rows(tile, r0, C::kBlocks);
-          fence_proxy_async_smem();
-        }
-      };
-      bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma) &&
-                mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma) &&
-                mbar_wait(x_ready, 0, abort_flag, a.status, kSiteMma);
-      if (ok) {
-        clear_padding(sK, sk - n0);
-        clear_padding(sV, sk - n0);
-        clear_padding(sQ, sq - mb * 128);
-        tc_fence_after();
-        bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ, hiK, idesc_kk);
-        mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
-        tc_commit(s_full);
-        ok = mbar_wait(do_full(0), 0, abort_flag, a.status, kSiteMma);
-      }
-      if (ok) {
-        clear_padding(sDO, sq - mb * 128);
-        tc_fence_after();
-        bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO, hiK, idesc_kk);
-        mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
-        tc_commit(dp_full);
-      }
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int qs = it % C::kQStages, dos = it % C::kDOStages;
-        const int nx = it + 1, nqs = nx % C::kQStages, ndos = nx % C::kDOStages;
-        const uint32_t npar = (nx / C::kQStages) & 1, ndpar = (nx / C::kDOStages) & 1;
-        // dV += P^T dO  (P^T from TMEM, dO MN-major)
-        if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
-        tc_fence_after();
-        bwd_issue_ts_halves(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_acc,
-                            it > 0);
-        tc_commit(do_empty(dos));
-        if (nx < n_it) {
-          if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
-          clear_padding(sQ + nqs * C::kTileBytes, sq - (mb + nx) * 128);
+      // The issue loop is instantiated twice, with the padding clears (some
+      // side is padded) and without them, so dense and packed calls run code
+      // that carries no trace of the clears.
+      auto issue_all = [&](auto padding) {
+        // Padded batches: tile rows past seqlen_q / seqlen_k hold the caller's
+        // padding, not TMA zero fill; P and dS are 0 there, but 0 * NaN is not,
+        // so those rows are zeroed before the tensor cores first read a tile.
+        auto clear_padding = [&](bool side_padded, uint32_t tile, int r0) {
+          if constexpr (decltype(padding)::value) {
+            if (side_padded && r0 < 128) {
+              zero_tile_rows(tile, r0, C::kBlocks);
+              fence_proxy_async_smem();
+            }
+          } else {
+            (void)side_padded, (void)tile, (void)r0;
+          }
+        };
+        bool ok = mbar_wait(kv_full, 0, abort_flag, a.status, kSiteMma) &&
+                  mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma) &&
+                  mbar_wait(x_ready, 0, abort_flag, a.status, kSiteMma);
+        if (ok) {
+          clear_padding(a.k_padded, sK, sk - n0);
+          clear_padding(a.k_padded, sV, sk - n0);
+          clear_padding(a.q_padded, sQ, sq - mb * 128);
           tc_fence_after();
-          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ + nqs * kTile16, hiK, idesc_kk);
+          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ, hiK, idesc_kk);
           mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
           tc_commit(s_full);
+          ok = mbar_wait(do_full(0), 0, abort_flag, a.status, kSiteMma);
         }
-        // dK += dS^T Q
-        if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
-        tc_fence_after();
-        bwd_issue_ts_halves(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_acc,
-                            it > 0);
-        tc_commit(q_empty(qs));
-        // dQ tile (into the dP columns when aliased: in order after dK read them)
-        if (!C::kAliasDQ && it > 0 &&
-            !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag, a.status, kSiteMma)))
-          break;
-        if (C::kDqTransposed)
-          bwd_issue_mn(tmem + C::kColDQ, loKm, loDSm, hiM, idesc_dq);   // K^T dS^T
-        else
-          bwd_issue_mn(tmem + C::kColDQ, loDSm, loKm, hiM, idesc_dq);   // dS K
-        tc_commit(dq_mma);
-        if (nx < n_it) {
-          if (!(ok = mbar_wait(do_full(ndos), ndpar, abort_flag, a.status, kSiteMma))) break;
-          if (C::kAliasDQ && !(ok = mbar_wait(dq_free, it & 1, abort_flag, a.status, kSiteMma)))
-            break;
-          clear_padding(sDO + ndos * C::kTileBytes, sq - (mb + nx) * 128);
+        if (ok) {
+          clear_padding(a.q_padded, sDO, sq - mb * 128);
           tc_fence_after();
-          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + ndos * kTile16, hiK, idesc_kk);
+          bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO, hiK, idesc_kk);
           mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
           tc_commit(dp_full);
         }
-      }
-      tc_commit(acc_done);
+        for (int it = 0; it < n_it && ok; ++it) {
+          const int qs = it % C::kQStages, dos = it % C::kDOStages;
+          const int nx = it + 1, nqs = nx % C::kQStages, ndos = nx % C::kDOStages;
+          const uint32_t npar = (nx / C::kQStages) & 1, ndpar = (nx / C::kDOStages) & 1;
+          // dV += P^T dO  (P^T from TMEM, dO MN-major)
+          if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
+          tc_fence_after();
+          bwd_issue_ts_halves(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_acc,
+                              it > 0);
+          tc_commit(do_empty(dos));
+          if (nx < n_it) {
+            if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
+            clear_padding(a.q_padded, sQ + nqs * C::kTileBytes, sq - (mb + nx) * 128);
+            tc_fence_after();
+            bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ + nqs * kTile16, hiK, idesc_kk);
+            mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
+            tc_commit(s_full);
+          }
+          // dK += dS^T Q
+          if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
+          tc_fence_after();
+          bwd_issue_ts_halves(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_acc,
+                              it > 0);
+          tc_commit(q_empty(qs));
+          // dQ tile (into the dP columns when aliased: in order after dK read them)
+          if (!C::kAliasDQ && it > 0 &&
+              !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag, a.status, kSiteMma)))
+            break;
+          if (C::kDqTransposed)
+            bwd_issue_mn(tmem + C::kColDQ, loKm, loDSm, hiM, idesc_dq);   // K^T dS^T
+          else
+            bwd_issue_mn(tmem + C::kColDQ, loDSm, loKm, hiM, idesc_dq);   // dS K
+          tc_commit(dq_mma);
+          if (nx < n_it) {
+            if (!(ok = mbar_wait(do_full(ndos), ndpar, abort_flag, a.status, kSiteMma))) break;
+            if (C::kAliasDQ && !(ok = mbar_wait(dq_free, it & 1, abort_flag, a.status, kSiteMma)))
+              break;
+            clear_padding(a.q_padded, sDO + ndos * C::kTileBytes, sq - (mb + nx) * 128);
+            tc_fence_after();
+            bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + ndos * kTile16, hiK, idesc_kk);
+            mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
+            tc_commit(dp_full);
+          }
+        }
+        tc_commit(acc_done);
+      };
+      if (a.q_padded || a.k_padded)
+        issue_all(Flag<true>{});
+      else
+        issue_all(Flag<false>{});
     }
   }
   } else if (warp < 8) {
@@ -461,13 +479,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       if (i >= sq) return 0.f;
       if (half == 0) {
         int64_t li;
-        if (a.packed)
+        if (a.q_packed)
           li = a.lse_th ? (int64_t)(qrow0 + i) * a.H + h : (int64_t)h * a.total_q + qrow0 + i;
         else
           li = a.lse_th ? ((int64_t)b * a.Sq + i) * a.H + h : ((int64_t)b * a.H + h) * a.Sq + i;
         return a.lse[li];
       }
-      const int64_t row = a.packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
+      const int64_t row = a.q_packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
       return a.delta[(int64_t)h * a.rows + row];
     };
     // The per-query constants enter the products through the extra K step:
@@ -622,7 +640,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int32_t m0 = (mb + it) * 128;
-      const int64_t row0 = a.packed ? (int64_t)(qrow0 + m0) : (int64_t)b * a.Sq + m0;
+      const int64_t row0 = a.q_packed ? (int64_t)(qrow0 + m0) : (int64_t)b * a.Sq + m0;
       // Each warp stages 32 x 32 fp32 boxes (32 rows of the accumulator x 32
       // head-dim columns, 128-byte swizzled like the tensor map) in one of its
       // two buffers and adds them with a TMA bulk reduction.  Rows of queries

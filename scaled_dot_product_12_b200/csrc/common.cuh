@@ -379,6 +379,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+// A compile-time flag passed to generic lambdas (for `if constexpr` code
+// paths instantiated per call site).
+template <bool V>
+struct Flag {
+  static constexpr bool value = V;
+};
+
 // Zeroes rows [r0, 128) of a 128-row tile of 16-bit elements stored as
 // `blocks` 64-column blocks of 128-byte rows, 16 KiB apart (whole rows, so
 // the swizzle inside a row does not matter).  One thread; the caller fences

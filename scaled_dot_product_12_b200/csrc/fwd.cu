@@ -89,15 +89,22 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
   const int mblk = gridDim.x - 1 - blockIdx.x;  // longest causal rows first
   const int h = blockIdx.y;
   const int b = blockIdx.z;
-  int32_t sq = args.Sq, sk = args.Sk, qrow0 = 0, krow0 = 0, bcoord = b;
-  if (args.packed) {
+  // Q and K sides are addressed independently: packed (rows from the
+  // cumulative lengths, TMA batch coordinate 0), padded (dense rows, lengths
+  // from the per-batch array) or dense.
+  int32_t sq = args.Sq, sk = args.Sk, qrow0 = 0, krow0 = 0, bq = b, bk = b;
+  if (args.q_packed) {
     qrow0 = args.cu_q[b];
-    krow0 = args.cu_k[b];
     sq = args.cu_q[b + 1] - qrow0;
-    sk = args.cu_k[b + 1] - krow0;
-    bcoord = 0;
-  } else if (args.padded) {
+    bq = 0;
+  } else if (args.q_padded) {
     sq = min(max(args.cu_q[b], 0), args.Sq);
+  }
+  if (args.k_packed) {
+    krow0 = args.cu_k[b];
+    sk = args.cu_k[b + 1] - krow0;
+    bk = 0;
+  } else if (args.k_padded) {
     sk = min(max(args.cu_k[b], 0), args.Sk);
   }
   const int32_t m0 = mblk * 128 * NQ;
@@ -109,14 +116,14 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
 
   // Output addressing for row i (sequence-local) of this head.
   auto o_row_ptr = [&](int32_t i) -> uint8_t* {
-    int64_t off = args.packed ? (int64_t)(qrow0 + i) * args.o_stride[2]
+    int64_t off = args.q_packed ? (int64_t)(qrow0 + i) * args.o_stride[2]
                               : (int64_t)b * args.o_stride[0] + (int64_t)i * args.o_stride[2];
     off += (int64_t)h * args.o_stride[1];
     return reinterpret_cast<uint8_t*>(args.o) + 2 * off;
   };
   auto lse_ptr = [&](int32_t i) -> float* {
     int64_t idx;
-    if (args.packed)
+    if (args.q_packed)
       idx = args.lse_th ? (int64_t)(qrow0 + i) * args.H + h : (int64_t)h * args.total_q + qrow0 + i;
     else
       idx = args.lse_th ? ((int64_t)b * args.Sq + i) * args.H + h
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         mbar_expect_tx(q_full(t), C::kTileBytes);
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sQ + t * C::kTileBytes + blk * 16384, &args.tq, q_full(t), 64 * blk,
-                      qrow0 + m0 + 128 * t, h, bcoord);
+                      qrow0 + m0 + 128 * t, h, bq);
       }
       int issued = 0;
       for (int it = 0; it < n_tiles; ++it) {
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         mbar_expect_tx(k_full(ks), C::kTileBytes);
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sK + ks * C::kTileBytes + blk * 16384, &args.tk, k_full(ks), 64 * blk, krow,
-                      h, bcoord);
+                      h, bk);
         const int vs = it % C::kVStages, vr = it / C::kVStages;
         if (vr > 0 && !mbar_wait(v_empty(vs), (vr - 1) & 1, abort_flag, args.status, kSiteLoad)) {
           issued = 2 * it + 1;
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         mbar_expect_tx(v_full(vs), C::kTileBytes);
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sV + vs * C::kTileBytes + blk * 16384, &args.tv, v_full(vs), 64 * blk, krow,
-                      h, bcoord);
+                      h, bk);
         issued = 2 * it + 2;
       }
       if (*abort_flag) {
@@ -252,67 +259,80 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         ok = mbar_wait(q_full(t), 0, abort_flag, args.status, kSiteMma);
       // O_t (+)= P_t V: P from TMEM (16 columns of 32 bits per 16 keys... 8
       // columns per K step of 16 keys), V MN-major, next 16 keys = +2048 bytes.
-      // Padded batches: rows of a V tile past seqlen_k hold the caller's
-      // padding, not TMA zero fill; P is 0 there, but 0 * NaN is not, so the
-      // rows are zeroed before the tensor cores read the tile.
-      auto clear_v_padding = [&](int it_v) {
-        const int r0 = sk - (nb + it_v) * 128;
-        if (args.padded && r0 < 128) {
-          zero_tile_rows(sV + (it_v % C::kVStages) * C::kTileBytes, r0, C::kBlocks);
-          fence_proxy_async_smem();
+      // The issue loop is instantiated twice, with the V padding clears (K
+      // side padded) and without them, so other calls run code that carries
+      // no trace of the clears.
+      auto issue_all = [&](auto padding) {
+        // Padded batches: rows of a V tile past seqlen_k hold the caller's
+        // padding, not TMA zero fill; P is 0 there, but 0 * NaN is not, so the
+        // rows are zeroed before the tensor cores read the tile.
+        auto clear_v_padding = [&](int it_v) {
+          if constexpr (decltype(padding)::value) {
+            const int r0 = sk - (nb + it_v) * 128;
+            if (r0 < 128) {
+              zero_tile_rows(sV + (it_v % C::kVStages) * C::kTileBytes, r0, C::kBlocks);
+              fence_proxy_async_smem();
+            }
+          } else {
+            (void)it_v;
+          }
+        };
+        auto issue_pv = [=](int t, int it_prev) {
+          fwd_issue_pv(tmem + C::kColO + DPAD * t, tmem + 128 * t,
+                       dV + (uint32_t)(it_prev % C::kVStages) * kTile16, kHiV, idesc_o, it_prev > 0);
+          tc_commit(bar0 + 8 * (bs + 2 * NQ + t));  // o_done(t)
+        };
+        // S_t = Q_t K^T: both K-major; 16-column K steps are +32 bytes inside a
+        // 64-column block, blocks 16 KiB apart.  Padded head-dim columns are
+        // zero in both operands (TMA fill), so all DPAD/16 steps are issued.
+        auto issue_s = [=](int t, int ks) {
+          fwd_issue_s<DPAD / 16>(tmem + 128 * t, dQ + (uint32_t)t * kTile16,
+                                 dK + (uint32_t)ks * kTile16, kHiK, idesc_s);
+          tc_commit(bar0 + 8 * (bs + t));  // s_full(t)
+        };
+        for (int it = 0; it < n_tiles && ok; ++it) {
+          const int ks = it % C::kKStages;
+          if (!(ok = mbar_wait(k_full(ks), (it / C::kKStages) & 1, abort_flag, args.status, kSiteMma)))
+            break;
+          for (int t = 0; t < NQ && ok; ++t) {
+            if (it > 0) {
+              if (!(ok = mbar_wait(p_ready(t), (it - 1) & 1, abort_flag, args.status, kSiteMma))) break;
+              if (t == 0) {
+                const int vs = (it - 1) % C::kVStages;
+                if (!(ok = mbar_wait(v_full(vs), ((it - 1) / C::kVStages) & 1, abort_flag,
+                                     args.status, kSiteMma)))
+                  break;
+                clear_v_padding(it - 1);
+              }
+              tc_fence_after();
+              issue_pv(t, it - 1);
+              if (t == NQ - 1) tc_commit(v_empty((it - 1) % C::kVStages));
+            }
+            issue_s(t, ks);
+          }
+          if (!ok) break;
+          tc_commit(k_empty(ks));
         }
-      };
-      auto issue_pv = [=](int t, int it_prev) {
-        fwd_issue_pv(tmem + C::kColO + DPAD * t, tmem + 128 * t,
-                     dV + (uint32_t)(it_prev % C::kVStages) * kTile16, kHiV, idesc_o, it_prev > 0);
-        tc_commit(bar0 + 8 * (bs + 2 * NQ + t));  // o_done(t)
-      };
-      // S_t = Q_t K^T: both K-major; 16-column K steps are +32 bytes inside a
-      // 64-column block, blocks 16 KiB apart.  Padded head-dim columns are
-      // zero in both operands (TMA fill), so all DPAD/16 steps are issued.
-      auto issue_s = [=](int t, int ks) {
-        fwd_issue_s<DPAD / 16>(tmem + 128 * t, dQ + (uint32_t)t * kTile16,
-                               dK + (uint32_t)ks * kTile16, kHiK, idesc_s);
-        tc_commit(bar0 + 8 * (bs + t));  // s_full(t)
-      };
-      for (int it = 0; it < n_tiles && ok; ++it) {
-        const int ks = it % C::kKStages;
-        if (!(ok = mbar_wait(k_full(ks), (it / C::kKStages) & 1, abort_flag, args.status, kSiteMma)))
-          break;
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (it > 0) {
-            if (!(ok = mbar_wait(p_ready(t), (it - 1) & 1, abort_flag, args.status, kSiteMma))) break;
+        if (ok) {
+          const int last = n_tiles - 1;
+          for (int t = 0; t < NQ && ok; ++t) {
+            if (!(ok = mbar_wait(p_ready(t), last & 1, abort_flag, args.status, kSiteMma))) break;
             if (t == 0) {
-              const int vs = (it - 1) % C::kVStages;
-              if (!(ok = mbar_wait(v_full(vs), ((it - 1) / C::kVStages) & 1, abort_flag,
-                                   args.status, kSiteMma)))
+              const int vs = last % C::kVStages;
+              if (!(ok = mbar_wait(v_full(vs), (last / C::kVStages) & 1, abort_flag, args.status,
+                                   kSiteMma)))
                 break;
-              clear_v_padding(it - 1);
+              clear_v_padding(last);
             }
             tc_fence_after();
-            issue_pv(t, it - 1);
-            if (t == NQ - 1) tc_commit(v_empty((it - 1) % C::kVStages));
+            issue_pv(t, last);
           }
-          issue_s(t, ks);
         }
-        if (!ok) break;
-        tc_commit(k_empty(ks));
-      }
-      if (ok) {
-        const int last = n_tiles - 1;
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (!(ok = mbar_wait(p_ready(t), last & 1, abort_flag, args.status, kSiteMma))) break;
-          if (t == 0) {
-            const int vs = last % C::kVStages;
-            if (!(ok = mbar_wait(v_full(vs), (last / C::kVStages) & 1, abort_flag, args.status,
-                                 kSiteMma)))
-              break;
-            clear_v_padding(last);
-          }
-          tc_fence_after();
-          issue_pv(t, last);
-        }
-      }
+      };
+      if (args.k_padded)
+        issue_all(Flag<true>{});
+      else
+        issue_all(Flag<false>{});
       // Everything issued has completed before TMEM is released.
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, args.status, kSiteTeardown);

@@ -18,8 +18,11 @@ struct FwdArgs {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int32_t B, H, Sq, Sk, D;
-  int32_t wl, wr, bottom_right, packed, lse_th, bf16, negate;
-  int32_t padded;  // BHSD with per-batch lengths in cu_q / cu_k (B entries each)
+  int32_t wl, wr, bottom_right, lse_th, bf16, negate;
+  // Per side (Q: Q, O, LSE; K: K, V): packed 1THD with cumulative lengths in
+  // cu_q / cu_k (B + 1 entries), or padded BHSD with per-batch lengths (B
+  // entries); neither: dense BHSD.
+  int32_t q_packed, k_packed, q_padded, k_padded;
   int64_t total_q;
   float scale_log2;  // |sm_scale| * log2(e)
   uint32_t* status;
@@ -38,9 +41,10 @@ struct BwdArgs {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int32_t B, H, Sq, Sk, D;
-  int32_t wl, wr, bottom_right, packed, lse_th, bf16;
-  int32_t padded;  // BHSD with per-batch lengths in cu_q / cu_k (B entries each)
-  int64_t total_q, rows;  // rows of the workspace: B*Sq (dense) or total_q
+  int32_t wl, wr, bottom_right, lse_th, bf16;
+  // Per side, as in FwdArgs (Q: Q, O, LSE, dO, dQ; K: K, V, dK, dV).
+  int32_t q_packed, k_packed, q_padded, k_padded;
+  int64_t total_q, rows;  // rows of the workspace: B*Sq, or total_q when Q is packed
   float sm_scale;
   float scale_log2;       // sm_scale * log2(e) (sign kept)
   float* delta;           // workspace: [H][rows]

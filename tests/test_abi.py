@@ -93,7 +93,7 @@ def _call_fwd(B, p):
     ("B", -1), ("Sq", 1 << 30), ("sm_scale", float("nan")), ("sm_scale", float("inf")),
     ("varlen_bits", 1 << 19), ("varlen_bits", 1 << 31), ("varlen_bits", 0x20),
     ("varlen_bits", 0x2000), ("varlen_bits", 2 << 16), ("varlen_bits", 3 << 16),
-    ("varlen_bits", 0x0B),                       # packed Q with dense K
+    ("varlen_bits", 0x0B),                       # packed Q without cu_seqlens_q
     ("varlen_bits", 0x0505),                     # length = array: not supported
     ("q", 0), ("o", 0), ("k", 0), ("q", FAKE + 8), ("o", FAKE + 2),
     ("q_stride", (3 * 128 * 64, 128 * 64, 60)),  # row stride of 120 bytes

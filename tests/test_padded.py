@@ -62,10 +62,24 @@ def test_padded_mode_needs_both_length_arrays():
     assert B.lib().attn_fwd(ctypes.byref(p), None) == B.ERROR_INVALID_VALUE
 
 
-def test_padded_queries_with_dense_keys_rejected():
+def test_each_side_needs_its_own_length_array():
     B = binding()
-    for qm, km in ((B.MODE_PADDED, B.MODE_DENSE), (B.MODE_DENSE, B.MODE_PADDED),
-                   (B.MODE_PADDED, B.MODE_PACKED)):
+    fake = 0x7F0000000000
+    for qm, km, have_q, have_k in ((B.MODE_PADDED, B.MODE_DENSE, False, True),
+                                   (B.MODE_DENSE, B.MODE_PADDED, True, False),
+                                   (B.MODE_PACKED, B.MODE_PADDED, False, True),
+                                   (B.MODE_PADDED, B.MODE_PACKED, True, False)):
+        p = _fwd_params(B, B.varlen_bits(qm, km, 0, 0), with_lengths=False)
+        p.total_q = p.total_k = 100
+        p.cu_seqlens_q = fake if have_q else 0
+        p.cu_seqlens_k = fake if have_k else 0
+        assert B.lib().attn_fwd(ctypes.byref(p), None) == B.ERROR_INVALID_VALUE, (qm, km)
+
+
+@pytest.mark.parametrize("mode", [B_mode for B_mode in (0x05, 0x06, 0x10, 0x12, 0x0D)])
+def test_unknown_modes_rejected(mode):
+    B = binding()
+    for qm, km in ((mode, B.MODE_DENSE), (B.MODE_PADDED, mode)):
         p = _fwd_params(B, B.varlen_bits(qm, km, 0, 0), with_lengths=True)
         assert B.lib().attn_fwd(ctypes.byref(p), None) == B.ERROR_INVALID_VALUE
 
