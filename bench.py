@@ -343,15 +343,31 @@ def power_capped(clocks):
     return bool(mhz and top and mhz < 0.97 * top)
 
 
+KERNEL_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu", "bwd.cu")
+
+
+def kernels_sha256():
+    """Hash of the kernel sources, to tie committed counters to a kernel build."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "scaled_dot_product_12_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def load_traffic(kernel, workload):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if one
-    for this kernel and workload exists (else null)."""
+    for this kernel and workload exists and was taken on the kernel sources
+    built now (else null: counters of another build do not describe this one)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    return d.get(f"{kernel}:{workload}")
+    if d.get("kernels_sha256") != kernels_sha256():
+        return None
+    return d.get("bytes_per_launch", {}).get(f"{kernel}:{workload}")
 
 
 def run_e2e(step: Step, stream, dev, n, flops, world):
