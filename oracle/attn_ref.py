@@ -31,7 +31,7 @@ section "Bottom-Right Aligned Sliding Windows": a numeric window becomes
 L = wl - d, R = wr + d with d = seqlen_k - seqlen_q taken per sequence;
 sentinel windows are never shifted).
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
   * a row i may attend key j iff j >= i - L and j <= i + R, both ends
     inclusive, an unbounded side imposing nothing;
   * the causal sentinels name their own diagonal: CAUSAL_TOP_LEFT allows
