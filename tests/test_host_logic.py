@@ -1,0 +1,99 @@
+"""Host-side logic that needs no GPU: how the binding derives sizes and
+VarlenBits from the tensors it is given (each side dense, packed or padded),
+and the bench's choice of roofline denominator and helper-kernel bandwidth."""
+
+from __future__ import annotations
+
+import pytest
+import torch
+
+import bench
+from scaled_dot_product_12_b200 import binding as B
+from scaled_dot_product_12_b200 import synth
+
+
+def _t(*shape):
+    return torch.zeros(shape, dtype=torch.bfloat16)
+
+
+def _problem(q, k, **kw):
+    args = dict(cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None)
+    args.update(kw)
+    return B.Problem(q, k, None, (B.WINDOW_INF, B.WINDOW_INF), False, args["cu_seqlens_q"],
+                     args["cu_seqlens_k"], args["max_seqlen_q"], args["max_seqlen_k"], "HT",
+                     kw.get("seqlens_q"), kw.get("seqlens_k"))
+
+
+def test_dense_sizes_and_bits():
+    pr = _problem(_t(2, 3, 100, 64), _t(2, 3, 90, 64))
+    assert (pr.B, pr.H, pr.Sq, pr.Sk, pr.D) == (2, 3, 100, 90, 64)
+    assert pr.bits == 0 and pr.lse_shape() == (2, 3, 100)
+
+
+def test_packed_q_dense_k():
+    cu = synth.cumsum0([5, 7])
+    pr = _problem(_t(12, 3, 64), _t(2, 3, 90, 64), cu_seqlens_q=cu, max_seqlen_q=7)
+    assert (pr.B, pr.Sq, pr.Sk, pr.total_q, pr.total_k) == (2, 7, 90, 12, 0)
+    assert pr.bits == B.varlen_bits(B.MODE_PACKED, B.MODE_DENSE, 0, 0)
+    assert pr.lse_shape() == (3, 12)
+    assert pr.cu_q is cu and pr.cu_k is None
+
+
+def test_padded_q_packed_k():
+    lens = torch.tensor([3, 9], dtype=torch.int32)
+    cu_k = synth.cumsum0([4, 0])
+    pr = _problem(_t(2, 3, 9, 64), _t(4, 3, 64), seqlens_q=lens, cu_seqlens_k=cu_k,
+                  max_seqlen_k=4)
+    assert (pr.B, pr.Sq, pr.Sk, pr.total_q, pr.total_k) == (2, 9, 4, 0, 4)
+    assert pr.bits == B.varlen_bits(B.MODE_PADDED, B.MODE_PACKED, 0, 0)
+    assert pr.cu_q is lens and pr.cu_k is cu_k
+
+
+@pytest.mark.parametrize("kw,q,k", [
+    (dict(seqlens_q=torch.tensor([1, 2], dtype=torch.int32),
+          cu_seqlens_q=synth.cumsum0([1, 2]), max_seqlen_q=2), (3, 3, 64), (2, 3, 5, 64)),
+    (dict(cu_seqlens_q=synth.cumsum0([1, 2])), (3, 3, 64), (2, 3, 5, 64)),          # no max_seqlen
+    (dict(cu_seqlens_q=synth.cumsum0([1, 2, 3]), max_seqlen_q=3), (6, 3, 64), (2, 3, 5, 64)),
+    (dict(seqlens_k=torch.tensor([1, 2, 3], dtype=torch.int32)), (2, 3, 5, 64), (2, 3, 5, 64)),
+    (dict(), (3, 3, 64), (2, 3, 5, 64)),                                             # 3-D dense
+])
+def test_inconsistent_calls_rejected(kw, q, k):
+    with pytest.raises(ValueError):
+        _problem(_t(*q), _t(*k), **kw)
+
+
+def test_roofline_denominator_follows_the_clocks():
+    assert bench.power_capped({"reasons": ["sw_power_cap"], "sm_mhz": 1965, "sm_max_mhz": 1965})
+    assert bench.power_capped({"reasons": [], "sm_mhz": 1700, "sm_max_mhz": 1965})
+    assert not bench.power_capped({"reasons": [], "sm_mhz": 1950, "sm_max_mhz": 1965})
+    assert not bench.power_capped({"reasons": ["clocks not sampled"], "sm_mhz": None,
+                                   "sm_max_mhz": None})
+
+
+def test_helper_kernel_bytes():
+    w = synth.WORKLOADS["ltx_15300"]
+    d = bench.other_bandwidth(w, 1, 0.2, 6542.1)
+    rows = 15300 * 32
+    assert d["bytes"] == rows * (14 * 128 + 4)
+    assert d["gbs"] == pytest.approx(d["bytes"] / 0.2e-3 / 1e9, rel=1e-3)
+    assert d["frac"] == pytest.approx(d["gbs"] / 6542.1, rel=1e-3)
+    assert bench.other_bandwidth(w, 1, 0.0, 6542.1)["gbs"] is None
+
+
+def test_traffic_is_null_for_other_kernel_builds(tmp_path, monkeypatch):
+    import json
+    root = tmp_path
+    (root / "profiles").mkdir()
+    src = root / "scaled_dot_product_12_b200" / "csrc"
+    src.mkdir(parents=True)
+    for name in bench.KERNEL_SOURCES:
+        (src / name).write_text(name)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    good = bench.kernels_sha256()
+    table = {"attn_bwd_kernel:ltx_15300": 123}
+    (root / "profiles" / "traffic.json").write_text(
+        json.dumps({"kernels_sha256": good, "bytes_per_launch": table}))
+    assert bench.load_traffic("attn_bwd_kernel", "ltx_15300") == 123
+    assert bench.load_traffic("attn_fwd_kernel", "ltx_15300") is None
+    (src / "bwd.cu").write_text("changed")
+    assert bench.load_traffic("attn_bwd_kernel", "ltx_15300") is None
