@@ -9,15 +9,20 @@
 //  2. attn_bwd_kernel       one CTA per (128-key tile, head, sequence); it
 //                           keeps K, V and the dK, dV accumulators on chip and
 //                           walks the 128-query tiles whose window reaches its
-//                           keys: S^T = K Q^T, dP^T = V dO^T, P^T and
-//                           dS^T = P^T o (dP^T - delta) in TMEM, dV += P^T dO,
-//                           dK += dS^T Q, dQ_tile = dS K added into the fp32
-//                           accumulator.  dO has strides of its own (the 0.14b
-//                           notes, "Kernel Bug Fixes", record a kernel that
-//                           addressed dO with O's strides);
+//                           keys: S^T = K Q^T and dP^T = V dO^T, each with one
+//                           extra K step that subtracts the per-query
+//                           LSE*log2(e)/c resp. delta inside the product, P^T
+//                           and dS^T = P^T o (dP^T - delta) in TMEM,
+//                           dV += P^T dO, dK += dS^T Q, and the dQ tile added
+//                           into the fp32 accumulator by TMA bulk reductions.
+//                           dO has strides of its own (the 0.14b notes,
+//                           "Kernel Bug Fixes", record a kernel that addressed
+//                           dO with O's strides);
 //  3. attn_dq_convert_kernel  dQ = sm_scale * accumulator in the input dtype.
 // Warp roles of (2): warps 0-7 P / dS in two groups of query columns (one key
-// row per thread), warps 8-11 dQ drain, warp 12 TMA, warp 13 MMA.
+// row per thread) and the dK / dV epilogue, warps 8-11 dQ drain, warp 12 TMA,
+// warp 13 MMA, warps 14-15 idle (they complete the TMA/MMA warpgroup, whose
+// registers go to the others through setmaxnreg).
 #include <cuda_runtime.h>
 
 #include "common.cuh"

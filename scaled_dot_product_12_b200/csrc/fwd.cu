@@ -11,7 +11,9 @@
 //                    and the epilogue;
 //   warp 4*NQ        TMA producer: Q once, K and V through separate rings;
 //   warp 4*NQ+1      MMA issuer (one thread): S = Q K^T (smem x smem) and
-//                    O += P V (P from TMEM, V from smem), TMEM owner.
+//                    O += P V (P from TMEM, V from smem), TMEM owner;
+//   warps 4*NQ+2..   idle: they complete the producer / MMA warpgroup, whose
+//                    registers go to the softmax groups through setmaxnreg.
 // TMEM columns: S/P of tile t at [128 t, 128 t + 128), O of tile t at
 // [128 NQ + DPAD t, ...).
 #include <cuda_runtime.h>
