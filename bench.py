@@ -308,8 +308,8 @@ def run_gpu(args, rank, world, local):
                          "datasheet_dense": round(value / world / DATASHEET_DENSE_BF16_TFLOPS, 4)},
         "roofline": {"bound": "tensor", "kernel": dominant[0], "achieved": round(dominant[1], 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(dominant[1] / peak, 4),
-                     "peak_source": (f"{peak_src} bf16_tflops_sustained (the SM clock was "
-                                     "power-capped during the timed region)") if capped else
+                     "peak_source": (f"{peak_src} bf16_tflops_sustained (the power cap "
+                                     "lowered the SM clock in the timed region)") if capped else
                                     (f"{peak_src} bf16_tflops (burst: the SM clock stayed at "
                                      "its maximum during the timed region)"),
                      "traffic": traffic},
@@ -335,10 +335,10 @@ def other_bandwidth(w, world, ms, hbm_gbs):
 
 
 def power_capped(clocks):
-    """True if the clock record shows the power cap (or a median SM clock more
-    than 3% under the maximum) during the timed region."""
-    if "sw_power_cap" in clocks.get("reasons", []):
-        return True
+    """True if the power cap actually lowered the SM clock during the timed
+    region: a median SM clock more than 3 % under the maximum.  A cap flag
+    alone, with the clock still at its maximum, leaves the burst figure the
+    right denominator."""
     mhz, top = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
     return bool(mhz and top and mhz < 0.97 * top)
 

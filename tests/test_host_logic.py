@@ -63,7 +63,10 @@ def test_inconsistent_calls_rejected(kw, q, k):
 
 
 def test_roofline_denominator_follows_the_clocks():
-    assert bench.power_capped({"reasons": ["sw_power_cap"], "sm_mhz": 1965, "sm_max_mhz": 1965})
+    # a cap flag with the clock still at its maximum: burst figure
+    assert not bench.power_capped({"reasons": ["sw_power_cap"], "sm_mhz": 1965,
+                                   "sm_max_mhz": 1965})
+    assert bench.power_capped({"reasons": ["sw_power_cap"], "sm_mhz": 1755, "sm_max_mhz": 1965})
     assert bench.power_capped({"reasons": [], "sm_mhz": 1700, "sm_max_mhz": 1965})
     assert not bench.power_capped({"reasons": [], "sm_mhz": 1950, "sm_max_mhz": 1965})
     assert not bench.power_capped({"reasons": ["clocks not sampled"], "sm_mhz": None,
