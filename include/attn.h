@@ -39,8 +39,9 @@
  *     ATTN_ERROR_INVALID_VALUE (cudaErrorInvalidValue) for: a wrong
  *     struct_size / version, reserved VarlenBits set, an unsupported mode,
  *     dtype or head dimension, a NULL required pointer, a base address not
- *     16-byte aligned, a stride whose byte size is not a multiple of 16, or a
- *     backward workspace that is too small.  ATTN_ERROR_NO_KERNEL_IMAGE
+ *     16-byte aligned, a stride whose byte size is not a multiple of 16, a
+ *     backward workspace that is too small, or a backward with H * rows_q
+ *     (rows_q = B*Sq, or total_q for a packed Q side) of 2^31 - 256 or more.  ATTN_ERROR_NO_KERNEL_IMAGE
  *     (cudaErrorNoKernelImageForDevice) on a GPU other than sm_100.  Launch
  *     errors are passed through.  A failing call writes nothing.
  *   - Tensors: fp16 or bf16 (ATTN_DTYPE_*), the head dimension D contiguous

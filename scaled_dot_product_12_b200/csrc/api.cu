@@ -279,6 +279,9 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     if (rows_k > 0 && (!x || !aligned16(x))) return cudaErrorInvalidValue;
   if (rows_q > 0 && (!p->lse || (reinterpret_cast<uintptr_t>(p->lse) & 3u)))
     return cudaErrorInvalidValue;
+  // The dQ accumulator is reduced into through a 2-D tensor map whose row
+  // coordinate (head * rows + row) is a signed 32-bit TMA coordinate.
+  if ((int64_t)p->H * rows_q >= ((int64_t)1 << 31) - 256) return cudaErrorInvalidValue;
   const size_t ws = attn_bwd_workspace_size(p);
   if (ws > 0 && (!p->workspace || p->workspace_bytes < ws ||
                  (reinterpret_cast<uintptr_t>(p->workspace) & 255u)))

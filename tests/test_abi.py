@@ -140,6 +140,19 @@ def _bwd(lib_b, **kw):
     return p
 
 
+@pytest.mark.parametrize("kw", [
+    dict(H=3, B=1 << 20, Sq=1024),                                    # dense: 3 * 2^30 rows
+    dict(H=4, total_q=(1 << 29) + 64, total_k=300, cu_seqlens_q=FAKE, cu_seqlens_k=FAKE),
+])
+def test_backward_rejects_rows_past_the_tma_coordinate_range(B, kw):
+    # H * rows_q rows of the fp32 dQ accumulator are addressed by a signed
+    # 32-bit TMA coordinate: 2^31 - 256 or more is refused before any launch.
+    if "total_q" in kw:
+        kw = dict(kw, varlen_bits=B.varlen_bits(B.MODE_PACKED, B.MODE_PACKED, 0, 0))
+    p = _bwd(B, workspace_bytes=1 << 62, **kw)  # the workspace check alone would pass
+    assert B.lib().attn_bwd(ctypes.byref(p), None) == B.ERROR_INVALID_VALUE
+
+
 def test_workspace_size_formula(B):
     p = _bwd(B)
     n = 3 * 2 * 100
