@@ -35,7 +35,10 @@ import torch  # noqa: E402
 from scaled_dot_product_12_b200 import synth  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DATASHEET_DENSE_BF16_TFLOPS = 2250.0  # NVIDIA B200 dense fp16/bf16 (the 2:4-sparse figure halved)
+# NVIDIA's HGX B200 specification table gives FP16/BF16 tensor throughput as
+# 36 PFLOPS for the 8-GPU board, a figure stated with 2:4 structured sparsity;
+# per GPU and dense that is 36 / 8 / 2 = 2.25 PFLOPS.
+DATASHEET_DENSE_BF16_TFLOPS = 2250.0
 CLOCK_REASONS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
     0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -160,21 +163,73 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# workload
+# workload: sizes, allowed pairs and algorithmic bytes
 # ---------------------------------------------------------------------------
+def seqlens(w: synth.Workload):
+    """Per-sequence (seqlen_q, seqlen_k) lists of a workload."""
+    if w.packed:
+        return synth.varlen_seqlens(synth.VARLEN_SEQLEN_SEED)
+    return [w.Sq] * w.B, [w.Sk] * w.B
+
+
+def pair_count(sq: int, sk: int, wl: int, wr: int, bottom_right: bool) -> int:
+    """Allowed (query, key) pairs of one sequence, counted in closed form: row i
+    sees keys max(0, i - L) .. min(sk - 1, i + R) with (L, R) the window of the
+    AOTriton 0.15b release notes ("Bottom-Right Aligned Sliding Windows":
+    L = wl - d, R = wr + d under the bottom-right diagonal, d = sk - sq; the
+    causal sentinels mean (inf, 0) and (inf, d) and are never shifted).  This
+    is the benchmark's own count; the tests pin it to the oracle's mask."""
+    import numpy as np
+    if sq <= 0 or sk <= 0:
+        return 0
+    d = sk - sq
+    if wl == synth.CAUSAL_TOP_LEFT:
+        L, R = None, 0
+    elif wl == synth.CAUSAL_BOTTOM_RIGHT:
+        L, R = None, d
+    else:
+        L = None if wl == synth.WINDOW_INF else (wl - d if bottom_right else wl)
+        R = None if wr == synth.WINDOW_INF else (wr + d if bottom_right else wr)
+    i = np.arange(sq, dtype=np.int64)
+    lo = np.zeros(sq, dtype=np.int64) if L is None else np.maximum(i - L, 0)
+    hi = np.full(sq, sk - 1, dtype=np.int64) if R is None else np.minimum(i + R, sk - 1)
+    return int(np.maximum(hi - lo + 1, 0).sum())
+
+
 def workload_flops(w: synth.Workload):
-    from scaled_dot_product_12_b200 import binding as B
-    pairs = B.allowed_pairs(w.Sq, w.Sk, w.window_left, w.window_right, w.bottom_right)
-    n = pairs * w.B * w.H
+    """(forward FLOP, backward FLOP, allowed pairs) of one step on one GPU."""
+    sq, sk = seqlens(w)
+    n = w.H * sum(pair_count(a, b, w.window_left, w.window_right, w.bottom_right)
+                  for a, b in zip(sq, sk))
     return 4 * w.D * n, 10 * w.D * n, n
 
 
+def workload_bytes(w: synth.Workload):
+    """Algorithmic HBM bytes of one launch of each kernel (every tensor read or
+    written once; 16-bit Q, K, V, O, dO, dQ, dK, dV, fp32 LSE, delta and dQ
+    accumulator).  Per (query row, head): forward Q + O (4D) + LSE (4); main
+    backward Q + dO (4D), LSE + delta (8), accumulator read + write (8D);
+    preprocess + conversion 14D + 4.  Per (key row, head): forward K + V (4D);
+    main backward K + V + dK + dV (8D)."""
+    sq, sk = seqlens(w)
+    rq, rk, D = w.H * sum(sq), w.H * sum(sk), w.D
+    return {"attn_fwd_kernel": rq * (4 * D + 4) + rk * 4 * D,
+            "attn_bwd_kernel": rq * (12 * D + 8) + rk * 8 * D,
+            "bwd_other": rq * (14 * D + 4)}
+
+
 def describe(w: synth.Workload):
+    sq, sk = seqlens(w)
+    layout = ("packed 1THD with cumulative seqlens, LSE TH" if w.packed
+              else f"BHSD dense, LSE {'TH' if w.lse_th else 'HT'}")
+    per_tensor = w.H * sum(sq) * w.D * 2
     return {"workload": f"{w.name}: {w.describe}, fwd+bwd", "B": w.B, "H": w.H, "Sq": w.Sq,
-            "Sk": w.Sk, "D": w.D, "dtype": w.dtype,
-            "window": [w.window_left, w.window_right], "layout": "BHSD dense, LSE HT",
-            "l2": "inputs larger than L2 (Q, K, V, O, dO, dQ, dK, dV each "
-                  f"{w.B * w.H * w.Sq * w.D * 2 / 1e6:.0f} MB; L2 is 126 MB)"}
+            "Sk": w.Sk, "D": w.D, "dtype": w.dtype, "total_q": sum(sq), "total_k": sum(sk),
+            "window": [w.window_left, w.window_right],
+            "diagonal": "bottom-right" if w.bottom_right else "top-left", "layout": layout,
+            "l2": "working set larger than L2 (Q, O, dO, dQ each "
+                  f"{per_tensor / 1e6:.0f} MB, K, V, dK, dV each "
+                  f"{w.H * sum(sk) * w.D * 2 / 1e6:.0f} MB; L2 is 126 MB)"}
 
 
 class Step:
@@ -185,18 +240,32 @@ class Step:
         self.B = B
         self.w = w
         dtype = synth.DTYPES[w.dtype]
-        q, k, v, do = synth.qkv_do((w.B, w.H, w.Sq, w.D), (w.B, w.H, w.Sk, w.D), w.seed, dtype)
-        self.host = {"q": q, "k": k, "v": v, "do": do}
+        if w.packed:
+            sq, sk = seqlens(w)
+            cu_q, cu_k = synth.cumsum0(sq), synth.cumsum0(sk)
+            q, k, v, do = synth.qkv_do((int(cu_q[-1]), w.H, w.D), (int(cu_k[-1]), w.H, w.D),
+                                       w.seed, dtype)
+            self.host = {"q": q, "k": k, "v": v, "do": do, "cu_q": cu_q, "cu_k": cu_k}
+            self.cu_q, self.cu_k = cu_q.to(dev), cu_k.to(dev)
+            self.kw = dict(cu_seqlens_q=self.cu_q, cu_seqlens_k=self.cu_k, max_seqlen_q=max(sq),
+                           max_seqlen_k=max(sk), lse_layout="TH")
+        else:
+            q, k, v, do = synth.qkv_do((w.B, w.H, w.Sq, w.D), (w.B, w.H, w.Sk, w.D), w.seed, dtype)
+            self.host = {"q": q, "k": k, "v": v, "do": do}
+            self.cu_q = self.cu_k = None
+            self.kw = dict(lse_layout="TH" if w.lse_th else "HT")
         self.q, self.k, self.v, self.do = (t.to(dev) for t in (q, k, v, do))
         self.scale = w.D ** -0.5
         self.window = (w.window_left, w.window_right)
         self.o = torch.empty_like(self.q)
-        self.lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+        pr = B.Problem(self.q, self.k, self.scale, self.window, w.bottom_right,
+                       self.kw.get("cu_seqlens_q"), self.kw.get("cu_seqlens_k"),
+                       self.kw.get("max_seqlen_q"), self.kw.get("max_seqlen_k"),
+                       self.kw["lse_layout"])
+        self.lse = torch.empty(pr.lse_shape(), dtype=torch.float32, device=dev)
         self.dq = torch.empty_like(self.q)
         self.dk = torch.empty_like(self.k)
         self.dv = torch.empty_like(self.v)
-        pr = B.Problem(self.q, self.k, self.scale, self.window, w.bottom_right, None, None, None,
-                       None, "HT")
         self.bp = B.bwd_params(self.do, self.q, self.k, self.v, self.o, self.lse, pr, self.dq,
                                self.dk, self.dv)
         self.ws = torch.empty(max(1, B.workspace_bytes(self.bp)), dtype=torch.uint8, device=dev)
@@ -210,7 +279,8 @@ class Step:
         if ev is not None:
             ev[0].record(stream)
         B.forward(self.q, self.k, self.v, sm_scale=self.scale, window=self.window,
-                  bottom_right=self.w.bottom_right, out=self.o, lse=self.lse, stream=stream)
+                  bottom_right=self.w.bottom_right, out=self.o, lse=self.lse, stream=stream,
+                  **self.kw)
         if ev is not None:
             ev[1].record(stream)
             self.bp.main_kernel_events[0] = ev[2].cuda_event
@@ -221,14 +291,29 @@ class Step:
         B._check("attn_bwd", B.lib().attn_bwd(ctypes.byref(self.bp), stream.cuda_stream))
 
 
+def kernel_roofline(name, flops, nbytes, ms, peak_tflops, hbm_gbs):
+    """Achieved rate of one kernel against the roofline that bounds it: the
+    tensor pipe when flops / peak exceeds bytes / bandwidth, else HBM."""
+    t_tensor = flops / (peak_tflops * 1e12)
+    t_hbm = nbytes / (hbm_gbs * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "kernel": name, "achieved": round(ach, 1), "peak": peak_tflops,
+                "unit": "TFLOP/s", "frac": round(ach / peak_tflops, 4)}
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": name, "achieved": round(ach, 1), "peak": hbm_gbs,
+            "unit": "GB/s", "frac": round(ach / hbm_gbs, 4)}
+
+
 def run_gpu(args, rank, world, local):
     from scaled_dot_product_12_b200 import binding as B
-    w = synth.WORKLOADS[args.workload]
+    w = synth.ALL_WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     step = Step(w, dev)
     stream = torch.cuda.Stream(dev)
     fwd_flops, bwd_flops, pairs = workload_flops(w)
+    nbytes = workload_bytes(w)
     flops = fwd_flops + bwd_flops
     peaks, peak_src = load_peaks()
 
@@ -268,21 +353,31 @@ def run_gpu(args, rank, world, local):
     total_flops = sum_over_ranks(flops, world)
     value = total_flops / (ms_step * 1e-3) / 1e12
     # The denominator follows the clocks seen in the timed region: the burst
-    # GEMM figure while the SM clock stayed at its maximum, the sustained
-    # (power-capped) one once the power cap lowered it.  Both fractions are
-    # reported.
+    # GEMM figure while the SM clock stayed at its maximum, the sustained one
+    # once the clock was lowered.  Both fractions are reported.
     burst = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
     sustained = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
-    capped = power_capped(clock_summary)
-    peak = sustained if capped else burst
+    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    lowered = clock_lowered(clock_summary)
+    peak = sustained if lowered else burst
     fwd_tf = fwd_flops / (fwd_ms * 1e-3) / 1e12
     bwd_tf = bwd_flops / (main_ms * 1e-3) / 1e12
-    dominant = ("attn_bwd_kernel", bwd_tf, main_ms) if main_ms >= fwd_ms else ("attn_fwd_kernel",
-                                                                              fwd_tf, fwd_ms)
-    traffic = load_traffic(dominant[0], w.name)
+    if main_ms >= fwd_ms:
+        roof = kernel_roofline("attn_bwd_kernel", bwd_flops, nbytes["attn_bwd_kernel"], main_ms,
+                               peak, hbm)
+    else:
+        roof = kernel_roofline("attn_fwd_kernel", fwd_flops, nbytes["attn_fwd_kernel"], fwd_ms,
+                               peak, hbm)
+    roof["peak_source"] = peak_source(peak_src, lowered, clock_summary)
+    roof["traffic"] = load_traffic(roof["kernel"], w.name)
 
     # ---- end to end through the C ABI with host buffers ----
     e2e = run_e2e(step, stream, dev, min(args.steps, 5), flops, world)
+
+    def per_kernel(tf, ms, nb):
+        return {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4),
+                "frac_of_burst": round(tf / burst, 4), "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                "frac_of_hbm": round(nb / (ms * 1e-3) / 1e9 / hbm, 4)}
 
     line = {
         "metric": "attention TFLOP/s (fwd+bwd, unmasked FLOPs)", "value": round(value, 2),
@@ -291,28 +386,17 @@ def run_gpu(args, rank, world, local):
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
         "data": "synthetic: i.i.d. N(0,1) Q, K, V, dO from a fixed seed",
         "config": describe(w),
-        "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tf, 1),
-                "frac_of_peak": round(fwd_tf / peak, 4),
-                "frac_of_burst": round(fwd_tf / burst, 4)},
-        "bwd_main": {"ms": round(main_ms, 4), "tflops": round(bwd_tf, 1),
-                     "frac_of_peak": round(bwd_tf / peak, 4),
-                     "frac_of_burst": round(bwd_tf / burst, 4)},
+        "fwd": per_kernel(fwd_tf, fwd_ms, nbytes["attn_fwd_kernel"]),
+        "bwd_main": per_kernel(bwd_tf, main_ms, nbytes["attn_bwd_kernel"]),
         "bwd_other_ms": round(ms_step - fwd_ms - main_ms, 4),
         # The delta preprocess and the dQ conversion are HBM-bound: their
         # algorithmic bytes over the rest of the step (both kernels and the
         # gaps between launches) give a lower bound on their bandwidth.
-        "bwd_other": other_bandwidth(w, world, ms_step - fwd_ms - main_ms,
-                                     peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])),
+        "bwd_other": other_bandwidth(nbytes["bwd_other"] * world, ms_step - fwd_ms - main_ms, hbm),
         "frac_of_peak": {"measured_burst": round(value / world / burst, 4),
                          "measured_sustained": round(value / world / sustained, 4),
                          "datasheet_dense": round(value / world / DATASHEET_DENSE_BF16_TFLOPS, 4)},
-        "roofline": {"bound": "tensor", "kernel": dominant[0], "achieved": round(dominant[1], 1),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(dominant[1] / peak, 4),
-                     "peak_source": (f"{peak_src} bf16_tflops_sustained (the power cap "
-                                     "lowered the SM clock in the timed region)") if capped else
-                                    (f"{peak_src} bf16_tflops (burst: the SM clock stayed at "
-                                     "its maximum during the timed region)"),
-                     "traffic": traffic},
+        "roofline": roof,
         "gpu_launches": 4 * args.steps,
         "clocks": clock_summary,
         "e2e": e2e,
@@ -323,24 +407,32 @@ def run_gpu(args, rank, world, local):
     return line
 
 
-def other_bandwidth(w, world, ms, hbm_gbs):
+def other_bandwidth(nbytes, ms, hbm_gbs):
     """Preprocess reads O, dO (2 x 2D bytes per row and head) and writes delta
     (4) and the zeroed fp32 dQ accumulator (4D); the conversion reads the
     accumulator (4D) and writes dQ (2D): (14 D + 4) bytes per row and head."""
-    rows = w.B * w.Sq * w.H  # the bench workloads are dense
-    nbytes = rows * (14 * w.D + 4) * world
     gbs = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
     return {"ms": round(ms, 4), "bytes": nbytes, "gbs": round(gbs, 1) if gbs else None,
             "peak_gbs": hbm_gbs, "frac": round(gbs / hbm_gbs, 4) if gbs else None}
 
 
-def power_capped(clocks):
-    """True if the power cap actually lowered the SM clock during the timed
-    region: a median SM clock more than 3 % under the maximum.  A cap flag
+def clock_lowered(clocks):
+    """True if the SM clock was lowered during the timed region, whatever the
+    cause: a median SM clock more than 3 % under the maximum.  A throttle flag
     alone, with the clock still at its maximum, leaves the burst figure the
     right denominator."""
     mhz, top = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
     return bool(mhz and top and mhz < 0.97 * top)
+
+
+def peak_source(src, lowered, clocks):
+    if not lowered:
+        return (f"{src} bf16_tflops (burst: the SM clock stayed at its maximum during the "
+                "timed region)")
+    seen = [r for r in clocks.get("reasons", []) if r not in ("gpu_idle",)]
+    return (f"{src} bf16_tflops_sustained (median SM clock {clocks.get('sm_mhz')} MHz against "
+            f"a {clocks.get('sm_max_mhz')} MHz maximum; throttle reasons seen: "
+            f"{', '.join(seen) if seen else 'none'})")
 
 
 KERNEL_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu", "bwd.cu")
@@ -370,35 +462,98 @@ def load_traffic(kernel, workload):
     return d.get("bytes_per_launch", {}).get(f"{kernel}:{workload}")
 
 
-def run_e2e(step: Step, stream, dev, n, flops, world):
-    """The same step through the C ABI with pinned HOST inputs and outputs: H2D
-    of Q, K, V, dO and D2H of O, LSE, dQ, dK, dV inside the timed region."""
+def e2e_groups(w: synth.Workload, n_groups: int):
+    """Slices along which the end-to-end step is pipelined: batches when there
+    are several (LSE rows of a batch are contiguous in HT layout), else heads
+    of the single batch; packed workloads run as one group."""
+    if w.packed or n_groups <= 1:
+        return None, [slice(None)]
+    dim, size = (0, w.B) if w.B > 1 else (1, w.H)
+    n = min(n_groups, size)
+    edges = [size * g // n for g in range(n + 1)]
+    return dim, [slice(edges[g], edges[g + 1]) for g in range(n) if edges[g + 1] > edges[g]]
+
+
+def run_e2e(step: Step, stream, dev, n, flops, world, n_groups: int = 4):
+    """The same work through the same C-ABI calls from pinned HOST buffers:
+    every step copies Q, K, V, dO (and the cumulative seqlens of packed inputs)
+    in and O, LSE, dQ, dK, dV out inside the timed region.  Dense workloads
+    are cut into groups of batches (or of heads when B = 1), each a forward and
+    backward call of its own, and pipelined over three streams: group g's
+    inputs copy in while group g - 1 computes and group g - 2's outputs copy
+    out."""
+    w = step.w
+    B = step.B
     host_in = {k: v.pin_memory() for k, v in step.host.items()}
     outs = ["o", "lse", "dq", "dk", "dv"]
     host_out = {k: torch.empty(getattr(step, k).shape, dtype=getattr(step, k).dtype,
                                pin_memory=True) for k in outs}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    dim, groups = e2e_groups(w, n_groups)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def part(t, g):
+        if dim is None:
+            return t
+        return t[g] if dim == 0 else t[:, g]
+
+    kw = dict(sm_scale=step.scale, window=step.window, bottom_right=w.bottom_right, **step.kw)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    done_in = [ev() for _ in groups]
+    done_fb = [ev() for _ in groups]
+    done_out = [ev() for _ in groups]
+    started = [False] * len(groups)
+
+    def one_step():
+        for gi, g in enumerate(groups):
+            with torch.cuda.stream(s_in):
+                if started[gi]:
+                    s_in.wait_event(done_fb[gi])  # last step's compute no longer reads them
+                for name, t in host_in.items():
+                    dst = getattr(step, name)
+                    if name in ("cu_q", "cu_k"):
+                        dst.copy_(t, non_blocking=True)
+                    else:
+                        part(dst, g).copy_(part(t, g), non_blocking=True)
+                done_in[gi].record(s_in)
+            with torch.cuda.stream(stream):
+                stream.wait_event(done_in[gi])
+                if started[gi]:
+                    stream.wait_event(done_out[gi])  # last step's outputs have left
+                o, lse = part(step.o, g), part(step.lse, g)
+                q, k, v, do = (part(getattr(step, x), g) for x in ("q", "k", "v", "do"))
+                B.forward(q, k, v, out=o, lse=lse, stream=stream, **kw)
+                B.backward(do, q, k, v, o, lse, dq=part(step.dq, g), dk=part(step.dk, g),
+                           dv=part(step.dv, g), workspace=step.ws, stream=stream, **kw)
+                done_fb[gi].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_fb[gi])
+                for name in outs:
+                    part(host_out[name], g).copy_(part(getattr(step, name), g), non_blocking=True)
+                done_out[gi].record(s_out)
+            started[gi] = True
+
+    one_step()  # warm-up: the same work, untimed
+    torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for _ in range(n):
-            step.q.copy_(host_in["q"], non_blocking=True)
-            step.k.copy_(host_in["k"], non_blocking=True)
-            step.v.copy_(host_in["v"], non_blocking=True)
-            step.do.copy_(host_in["do"], non_blocking=True)
-            step.run(stream)
-            for k in outs:
-                host_out[k].copy_(getattr(step, k), non_blocking=True)
-        t1.record(stream)
+    t0.record(s_in)
+    for _ in range(n):
+        one_step()
+    s_out.wait_stream(stream)
+    s_out.wait_stream(s_in)
+    t1.record(s_out)
     torch.cuda.synchronize(dev)
     barrier(world)
     ms = max_over_ranks(t0.elapsed_time(t1) / n, world)
     total = sum_over_ranks(flops, world)
     return {"value": round(total / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipeline": (f"{len(groups)} groups of {'batches' if dim == 0 else 'heads'} over "
+                         "copy-in, compute and copy-out streams") if dim is not None
+            else "one group (copy in, compute, copy out in order)"}
 
 
 # ---------------------------------------------------------------------------
@@ -414,37 +569,44 @@ def _blas_threads():
 
 
 def oracle_sample(w: synth.Workload, rows: int):
-    """Inputs of a bounded sample: head (0, 0), the first `rows` query rows
-    (all rows if rows <= 0) against all keys, and its FLOP count."""
+    """Inputs of a bounded sample and its FLOP count (14*D per allowed pair,
+    counted with the oracle's own mask): head 0 of the first (batch or packed)
+    sequence, its first `rows` query rows (all rows if rows <= 0) against all
+    of its keys.  A prefix of the query rows is itself a problem with the same
+    mask rows only when the window does not depend on seqlen_q (top-left
+    windows, no mask); otherwise the whole sequence is the sample."""
     import numpy as np
+
+    from oracle import attn_ref as ref
     dtype = synth.DTYPES[w.dtype]
-    q, k, v, do = synth.qkv_do((w.B, w.H, w.Sq, w.D), (w.B, w.H, w.Sk, w.D), w.seed, dtype)
-    f = lambda t: t[0, 0].float().numpy().astype(np.float64)  # noqa: E731
-    qn, kn, vn, don = f(q), f(k), f(v), f(do)
-    if rows > 0:
-        qn, don = qn[:rows], don[:rows]
-    from scaled_dot_product_12_b200 import binding as B
-    pairs = B.allowed_pairs(qn.shape[0], w.Sk, w.window_left, w.window_right, w.bottom_right) \
-        if rows <= 0 or w.window_left == synth.WINDOW_INF and w.window_right == synth.WINDOW_INF \
-        else None
-    if pairs is None:
-        from oracle import attn_ref as ref
-        m = ref.allowed(w.Sq, w.Sk, w.window_left, w.window_right, w.bottom_right,
-                        rows=list(range(qn.shape[0])))
-        pairs = int(m.sum())
+    sq, sk = seqlens(w)
+    if w.packed:
+        q, k, v, do = synth.qkv_do((sum(sq), w.H, w.D), (sum(sk), w.H, w.D), w.seed, dtype)
+        f = lambda t, n: t[:n, 0].float().numpy().astype(np.float64)  # noqa: E731
+        qn, kn, vn, don = f(q, sq[0]), f(k, sk[0]), f(v, sk[0]), f(do, sq[0])
+    else:
+        q, k, v, do = synth.qkv_do((w.B, w.H, w.Sq, w.D), (w.B, w.H, w.Sk, w.D), w.seed, dtype)
+        f = lambda t: t[0, 0].float().numpy().astype(np.float64)  # noqa: E731
+        qn, kn, vn, don = f(q), f(k), f(v), f(do)
+    no_mask = w.window_left == synth.WINDOW_INF and w.window_right == synth.WINDOW_INF
+    depends_on_sq = w.window_left == synth.CAUSAL_BOTTOM_RIGHT or (
+        w.bottom_right and w.window_left != synth.CAUSAL_TOP_LEFT and not no_mask)
+    n = qn.shape[0] if rows <= 0 or depends_on_sq else min(rows, qn.shape[0])
+    qn, don = qn[:n], don[:n]
+    pairs = ref.allowed_count(n, kn.shape[0], w.window_left, w.window_right, w.bottom_right)
     return (qn, kn, vn, don), 14 * w.D * pairs
 
 
 def oracle_step(w, inputs):
-    """One oracle forward and backward; returns their wall times (s)."""
+    """One oracle forward and backward of the sample; returns their wall
+    times (s)."""
     from oracle import attn_ref as ref
     qn, kn, vn, don = inputs
-    # rows of a prefix keep their own mask only when the window does not
-    # depend on seqlen_q; the default workloads are unmasked or top-left.
+    args = (w.D ** -0.5, w.window_left, w.window_right, w.bottom_right)
     t0 = time.perf_counter()
-    ref.forward(qn, kn, vn, w.D ** -0.5, w.window_left, w.window_right, w.bottom_right)
+    ref.forward(qn, kn, vn, *args)
     t1 = time.perf_counter()
-    ref.backward(qn, kn, vn, don, w.D ** -0.5, w.window_left, w.window_right, w.bottom_right)
+    ref.backward(qn, kn, vn, don, *args)
     return t1 - t0, time.perf_counter() - t1
 
 
@@ -457,15 +619,15 @@ def cpu_baseline(w: synth.Workload, rows: int = 0):
             "kind": "oracle", "cpu_count": os.cpu_count(),
             "fwd_tflops": round(4 * w.D * pair_flops / t_f / 1e12, 6),
             "bwd_tflops": round(10 * w.D * pair_flops / t_b / 1e12, 6),
-            "sample": f"fp64 NumPy oracle, forward + backward of head (0,0) "
-                      f"({'all' if rows <= 0 else rows} query rows x {w.Sk} keys, "
-                      f"{flops / 1e9:.1f} GFLOP at 14*D per pair), {dt:.1f} s on "
+            "sample": f"fp64 NumPy oracle, forward + backward of head 0 of the first sequence "
+                      f"({inputs[0].shape[0]} query rows x {inputs[1].shape[0]} keys, "
+                      f"{flops / 1e9:.1f} GFLOP at 14*D per allowed pair), {dt:.1f} s on "
                       f"{os.cpu_count()} host cores"}
 
 
 def run_reference(args, rank, world):
     """--impl reference: the oracle as it stands, timed on the host cores."""
-    w = synth.WORKLOADS[args.workload]
+    w = synth.ALL_WORKLOADS[args.workload]
     rows = 256
     inputs, flops = oracle_sample(w, rows)
     for _ in range(args.warmup):
@@ -478,8 +640,9 @@ def run_reference(args, rank, world):
     dt = (time.perf_counter() - t) / args.steps
     pair_flops = flops / (14 * w.D)
     value = flops / dt / 1e12
-    sample = (f"each step: fp64 NumPy oracle forward + backward of head (0,0), first {rows} "
-              f"query rows against all {w.Sk} keys ({flops / 1e9:.2f} GFLOP)")
+    sample = (f"each step: fp64 NumPy oracle forward + backward of head 0 of the first sequence, "
+              f"its first {inputs[0].shape[0]} query rows against all {inputs[1].shape[0]} keys "
+              f"({flops / 1e9:.2f} GFLOP)")
     return {"impl": "reference", "metric": "attention TFLOP/s (fwd+bwd, unmasked FLOPs)",
             "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
@@ -499,7 +662,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="ltx_15300", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="ltx_15300", choices=sorted(synth.ALL_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

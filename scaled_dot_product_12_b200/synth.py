@@ -121,3 +121,24 @@ def varlen_cases(dims=(128, 48, 80)):
                 cases.append((f"varlen_D{D}_{tag}_{'BR' if br else 'TL'}", D, wl, wr, br, 9 + k))
                 k += 1
     return cases
+
+
+def varlen_workloads(dims=(128,)):
+    """The packed cases as named workloads: 16 sequences (lengths from
+    VARLEN_SEQLEN_SEED), H = 16, bf16, LSE in TH layout; Sq / Sk hold the
+    largest seqlen_q / seqlen_k."""
+    sq, sk = varlen_seqlens(VARLEN_SEQLEN_SEED)
+    out = {}
+    for name, D, wl, wr, br, seed in varlen_cases(dims):
+        win = {CAUSAL_TOP_LEFT: "causal top-left sentinel",
+               CAUSAL_BOTTOM_RIGHT: "causal bottom-right sentinel"}.get(wl, f"window ({wl}, {wr})")
+        out[name] = Workload(name, "bf16", len(sq), 16, max(sq), max(sk), D, wl, wr, br, seed,
+                             packed=True, lse_th=True,
+                             describe=(f"packed 1THD varlen, bf16 16 seqs (seqlen_q ~ U[1,4096], "
+                                       f"seqlen_k = seqlen_q + U[0,512]) H16 D{D}, {win}, "
+                                       f"{'bottom-right' if br else 'top-left'} diagonal, LSE TH"))
+    return out
+
+
+VARLEN_WORKLOADS = varlen_workloads()
+ALL_WORKLOADS = {**WORKLOADS, **VARLEN_WORKLOADS}

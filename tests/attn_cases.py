@@ -57,6 +57,40 @@ def rel_fro(a, b) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
+def local_blocks(a):
+    """Index tuples of the blocks whose error is also checked on its own: each
+    (b, h) and 128-row tile of a dense [B, H, S, D] tensor, each head and
+    128-token tile of a packed [T, H, D] tensor, each 128-row tile of a single
+    head [S, D]."""
+    a = np.asarray(a)
+    if a.ndim == 4:
+        return [(b, h, slice(r, r + 128)) for b in range(a.shape[0]) for h in range(a.shape[1])
+                for r in range(0, a.shape[2], 128)]
+    if a.ndim == 3:
+        return [(slice(r, r + 128), h) for h in range(a.shape[1]) for r in range(0, a.shape[0], 128)]
+    return [(slice(r, r + 128),) for r in range(0, a.shape[0], 128)]
+
+
+def local_errors(g, w):
+    """Per block: ||g - w|| / max(||w_block||, ||w|| * sqrt(n_block / n)).  The
+    floor is the norm an average block of that size would have, so a block
+    whose true gradient nearly cancels (a few allowed keys per row) is held to
+    an absolute error of TOL_GRAD times a typical block norm, while a wrong,
+    missing or zeroed block of ordinary size fails by a wide margin."""
+    g = np.asarray(g, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    total = np.linalg.norm(w)
+    out = []
+    for idx in local_blocks(w):
+        wb, gb = w[idx], g[idx]
+        if wb.size == 0:
+            continue
+        floor = total * np.sqrt(wb.size / w.size)
+        den = max(np.linalg.norm(wb), floor)
+        out.append((idx, float(np.linalg.norm(gb - wb) / den) if den > 0 else 0.0))
+    return out
+
+
 def assert_grads(got, want, what=""):
     for name, g, w in zip(("dQ", "dK", "dV"), got, want):
         g = np.asarray(g, dtype=np.float64)
@@ -70,6 +104,9 @@ def assert_grads(got, want, what=""):
             assert np.abs(g).max(initial=0.0) <= ZERO_GRAD_ABS, f"{what}: {name} should be 0"
         else:
             assert e <= TOL_GRAD, f"{what}: {name} relative Frobenius error {e}"
+            worst = max(local_errors(g, w), key=lambda t: t[1])
+            assert worst[1] <= TOL_GRAD, \
+                f"{what}: {name} block {worst[0]} relative Frobenius error {worst[1]}"
 
 
 def dense_inputs(B, H, Sq, Sk, D, dtype, seed):

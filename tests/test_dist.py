@@ -53,7 +53,10 @@ def _ref_worker(rank, world, port, out):
     with contextlib.redirect_stdout(buf):
         rc = bench.main(["--impl", "reference", "--workload", "tiny_causal", "--steps", "1",
                          "--warmup", "3"])
-    out[rank] = (rc, buf.getvalue())
+    # the reference arm runs the oracle alone: the product library stays unloaded
+    with open("/proc/self/maps") as f:
+        loaded = "libattn.so" in f.read()
+    out[rank] = (rc, buf.getvalue(), loaded)
 
 
 def test_reference_arm_prints_on_rank_zero_only():
@@ -67,3 +70,4 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert out[1][1] == ""
+    assert not out[0][2] and not out[1][2], "the reference arm loaded libattn.so"

@@ -63,24 +63,71 @@ def test_inconsistent_calls_rejected(kw, q, k):
 
 
 def test_roofline_denominator_follows_the_clocks():
-    # a cap flag with the clock still at its maximum: burst figure
-    assert not bench.power_capped({"reasons": ["sw_power_cap"], "sm_mhz": 1965,
-                                   "sm_max_mhz": 1965})
-    assert bench.power_capped({"reasons": ["sw_power_cap"], "sm_mhz": 1755, "sm_max_mhz": 1965})
-    assert bench.power_capped({"reasons": [], "sm_mhz": 1700, "sm_max_mhz": 1965})
-    assert not bench.power_capped({"reasons": [], "sm_mhz": 1950, "sm_max_mhz": 1965})
-    assert not bench.power_capped({"reasons": ["clocks not sampled"], "sm_mhz": None,
-                                   "sm_max_mhz": None})
+    # a throttle flag with the clock still at its maximum: burst figure
+    assert not bench.clock_lowered({"reasons": ["sw_power_cap"], "sm_mhz": 1965,
+                                    "sm_max_mhz": 1965})
+    assert bench.clock_lowered({"reasons": ["sw_power_cap"], "sm_mhz": 1755, "sm_max_mhz": 1965})
+    assert bench.clock_lowered({"reasons": [], "sm_mhz": 1700, "sm_max_mhz": 1965})
+    assert not bench.clock_lowered({"reasons": [], "sm_mhz": 1950, "sm_max_mhz": 1965})
+    assert not bench.clock_lowered({"reasons": ["clocks not sampled"], "sm_mhz": None,
+                                    "sm_max_mhz": None})
+    # the recorded source names the reasons that were actually seen
+    src = bench.peak_source("measured", True, {"sm_mhz": 1700, "sm_max_mhz": 1965,
+                                               "reasons": ["sw_thermal_slowdown"]})
+    assert "sw_thermal_slowdown" in src and "power cap" not in src
+    assert "none" in bench.peak_source("measured", True, {"sm_mhz": 1700, "sm_max_mhz": 1965,
+                                                          "reasons": []})
 
 
 def test_helper_kernel_bytes():
     w = synth.WORKLOADS["ltx_15300"]
-    d = bench.other_bandwidth(w, 1, 0.2, 6542.1)
+    nb = bench.workload_bytes(w)
     rows = 15300 * 32
-    assert d["bytes"] == rows * (14 * 128 + 4)
+    assert nb["bwd_other"] == rows * (14 * 128 + 4)
+    assert nb["attn_fwd_kernel"] == rows * (4 * 128 + 4) + rows * 4 * 128
+    assert nb["attn_bwd_kernel"] == rows * (12 * 128 + 8) + rows * 8 * 128
+    d = bench.other_bandwidth(nb["bwd_other"], 0.2, 6542.1)
     assert d["gbs"] == pytest.approx(d["bytes"] / 0.2e-3 / 1e9, rel=1e-3)
     assert d["frac"] == pytest.approx(d["gbs"] / 6542.1, rel=1e-3)
-    assert bench.other_bandwidth(w, 1, 0.0, 6542.1)["gbs"] is None
+    assert bench.other_bandwidth(nb["bwd_other"], 0.0, 6542.1)["gbs"] is None
+    # packed workloads count their tokens, not B * max_seqlen
+    wv = synth.VARLEN_WORKLOADS["varlen_D128_w256_0_TL"]
+    sq, sk = synth.varlen_seqlens(synth.VARLEN_SEQLEN_SEED)
+    assert bench.workload_bytes(wv)["bwd_other"] == 16 * sum(sq) * (14 * 128 + 4)
+    assert bench.workload_bytes(wv)["attn_fwd_kernel"] == \
+        16 * sum(sq) * (4 * 128 + 4) + 16 * sum(sk) * 4 * 128
+
+
+def test_kernel_roofline_picks_the_binding_resource():
+    r = bench.kernel_roofline("k", 1e12, 1e6, 1.0, 1000.0, 6000.0)   # AI 1e6: tensor
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(1000.0) and r["frac"] == pytest.approx(1.0)
+    r = bench.kernel_roofline("k", 1e9, 6e9, 1.0, 1000.0, 6000.0)    # AI 0.17: HBM
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(6000.0) and r["frac"] == pytest.approx(1.0)
+
+
+INF, CTL, CBR = synth.WINDOW_INF, synth.CAUSAL_TOP_LEFT, synth.CAUSAL_BOTTOM_RIGHT
+
+
+@pytest.mark.parametrize("w", [(INF, INF, 0), (CTL, 0, 0), (CTL, 0, 1), (CBR, 0, 0), (CBR, 0, 1),
+                               (INF, 0, 1), (256, 0, 0), (256, 0, 1), (-64, 128, 0),
+                               (-64, 128, 1), (3, -5, 0), (0, 0, 1), (-300, 200, 1),
+                               (130, INF, 1), (INF, -7, 0)])
+@pytest.mark.parametrize("sq,sk", [(1, 1), (5, 9), (128, 128), (200, 333), (333, 200),
+                                   (700, 513)])
+def test_bench_pair_count_matches_the_oracle_mask(w, sq, sk):
+    from oracle import attn_ref as ref
+    assert bench.pair_count(sq, sk, *w) == ref.allowed_count(sq, sk, *w)
+
+
+def test_bench_flops_of_the_packed_workload():
+    from oracle import attn_ref as ref
+    wv = synth.VARLEN_WORKLOADS["varlen_D128_w-64_128_BR"]
+    sq, sk = synth.varlen_seqlens(synth.VARLEN_SEQLEN_SEED)
+    want = 16 * sum(ref.allowed_count(a, b, -64, 128, True) for a, b in zip(sq, sk))
+    f, b, n = bench.workload_flops(wv)
+    assert n == want and f == 4 * 128 * n and b == 10 * 128 * n
 
 
 def test_traffic_is_null_for_other_kernel_builds(tmp_path, monkeypatch):
@@ -100,3 +147,16 @@ def test_traffic_is_null_for_other_kernel_builds(tmp_path, monkeypatch):
     assert bench.load_traffic("attn_fwd_kernel", "ltx_15300") is None
     (src / "bwd.cu").write_text("changed")
     assert bench.load_traffic("attn_bwd_kernel", "ltx_15300") is None
+
+
+def test_end_to_end_groups_cover_the_workload_once():
+    for name, w in synth.ALL_WORKLOADS.items():
+        dim, groups = bench.e2e_groups(w, 4)
+        if w.packed:
+            assert dim is None and groups == [slice(None)]
+            continue
+        size = w.B if dim == 0 else w.H
+        assert dim == (0 if w.B > 1 else 1)
+        covered = [i for g in groups for i in range(size)[g]]
+        assert covered == list(range(size)), name
+        assert 1 <= len(groups) <= 4

@@ -3,6 +3,10 @@
 * 0.14b notes, "Kernel Bug Fixes": an early-exit LSE write ran past a
   sequence under the stacked varlen layout -> canaries after the packed rows
   and around the head dimension stay untouched.
+* the same lesson for a cumulative-lengths array that runs past the packed
+  tensors (a caller's error): the sequences are clamped to the tensors, rows
+  past them (canaries) stay untouched and the rest matches the oracle on the
+  clamped lengths, forward and backward.
 * 0.14b notes, "Kernel Bug Fixes": a backward addressed dO with O's strides
   -> dO with a layout of its own gives the same gradients.
 * 0.15b notes, "Kernel Bug Fixes": the early-exit zero store was bounded by the
@@ -57,6 +61,47 @@ def test_packed_rows_past_the_last_sequence_stay_untouched(lse_layout, w):
     got_lse = lse_c.cpu().numpy()
     got_lse = got_lse.T if lse_layout == "TH" else got_lse
     assert_o_lse(o.float().cpu().numpy(), got_lse, want[0], want[1], torch.bfloat16)
+
+
+@pytest.mark.parametrize("w", [(INF, INF, False), (CTL, 0, False), (256, 0, True), (-64, 128, True)],
+                         ids=str)
+def test_cumulative_lengths_past_the_tensors_are_clamped(w):
+    B = binding()
+    dev = torch.device("cuda")
+    sq, sk = [130, 5, 257], [100, 300, 257]
+    H, D, pad = 2, 64, 300
+    q, k, v, do, cu_q, cu_k = packed_inputs(sq, sk, H, D, torch.bfloat16, 12)
+    tq, tk = sum(sq), sum(sk)
+    # the last entries claim 150 query rows and 200 key rows that do not exist
+    bad_q = cu_q.clone()
+    bad_q[-1] += 150
+    bad_k = cu_k.clone()
+    bad_k[-1] += 200
+    kw = dict(sm_scale=0.125, window=w[:2], bottom_right=w[2], cu_seqlens_q=bad_q.to(dev),
+              cu_seqlens_k=bad_k.to(dev), max_seqlen_q=257 + 150, max_seqlen_k=257 + 200,
+              lse_layout="TH")
+
+    def canary(rows):
+        buf = torch.full((rows + pad, H, D), NAN16, dtype=torch.bfloat16, device=dev)
+        return buf, buf[:rows]
+    o_buf, o = canary(tq)
+    dq_buf, dq = canary(tq)
+    dk_buf, dk = canary(tk)
+    dv_buf, dv = canary(tk)
+    lse_buf = torch.full((H * tq + pad,), float("nan"), device=dev)
+    lse = lse_buf[:H * tq].view(tq, H)
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    B.forward(qd, kd, vd, out=o, lse=lse, **kw)
+    B.backward(dod, qd, kd, vd, o, lse, dq=dq, dk=dk, dv=dv, **kw)
+    torch.cuda.synchronize()
+    assert B.device_status(dev) == 0
+    for buf, rows in ((o_buf, tq), (dq_buf, tq), (dk_buf, tk), (dv_buf, tk)):
+        assert torch.isnan(buf[rows:].float()).all(), "a write ran past the tensor"
+    assert torch.isnan(lse_buf[H * tq:]).all()
+    want = oracle_packed(q, k, v, do, cu_q, cu_k, 0.125, *w)
+    assert_o_lse(o.float().cpu().numpy(), lse.cpu().numpy().T, want["o"], want["lse_ht"],
+                 torch.bfloat16)
+    assert_grads([f64(t) for t in (dq, dk, dv)], [want["dq"], want["dk"], want["dv"]])
 
 
 @pytest.mark.parametrize("w", [(INF, INF, False), (0, -1, False), (CBR, 0, True)], ids=str)

@@ -144,3 +144,113 @@ def test_edge_probe_packed(w):
             want = hi if sign > 0 else lo
             assert np.array_equal(_decode(rows)[ne], want[ne]), (s, sign)
             assert np.all(rows[~ne] == 0)
+
+
+# ---------------------------------------------------------------------------
+# Backward edge probe.  Row i's scores are centred on the oracle's edge key
+# e(i) = hi(i) (or lo(i) with the sign flipped): S_ij = 32 (j - e(i)), exact
+# in fp16 / bf16 operands and in fp32.  If the backward admits exactly the
+# oracle's keys, P_i is one-hot on e(i) to within e^-32, and with
+# dO_i = unit vector (i mod 8), dV_j[c] is the number of rows i = c (mod 8)
+# whose edge key is j: an exact small integer.  A key the backward wrongly
+# admits past the edge would carry a positive score and take the weight; a
+# dropped edge key would move it inwards; either changes the counts.  V holds
+# base-16 digits of the key index, and O / LSE are the oracle's, so
+# dS = P o (dP - delta) vanishes wherever P is right: dQ and dK must be ~0.
+# Keys that no row may see get dK = dV = 0 exactly.
+# ---------------------------------------------------------------------------
+
+def _bwd_edge_inputs(sq, sk, D, dtype, edge, sign):
+    j = torch.arange(sk)
+    e = torch.as_tensor(np.maximum(edge, 0), dtype=torch.int64)
+    q = torch.zeros(sq, D)
+    q[:, 0], q[:, 1] = 2048.0 * sign, 32.0 * sign
+    q[:, 2], q[:, 3] = -2048.0 * sign * (e // 64).float(), -32.0 * sign * (e % 64).float()
+    k = torch.zeros(sk, D)
+    k[:, 0], k[:, 1], k[:, 2], k[:, 3] = (j // 64).float(), (j % 64).float(), 1.0, 1.0
+    v = torch.zeros(sk, D)
+    for c in range(4):
+        v[:, c] = ((j >> (4 * c)) & 15).float()
+    do = torch.zeros(sq, D)
+    do[torch.arange(sq), torch.arange(sq) % 8] = 1.0
+    return q.to(dtype), k.to(dtype), v.to(dtype), do.to(dtype)
+
+
+def _bwd_edge_expect(sq, sk, edge, cnt):
+    want = np.zeros((sk, 8))
+    for i in range(sq):
+        if cnt[i] > 0:
+            want[edge[i], i % 8] += 1
+    return want
+
+
+def _bwd_edge_run(B, q, k, v, do, w, dev, **kw):
+    """Forward on the oracle side (O rounded to the dtype, LSE in fp32), then
+    the GPU backward with those as its O and LSE."""
+    from attn_cases import f64
+    packed = "cu_seqlens_q" in kw
+    if packed:
+        cq, ck = kw["cu_seqlens_q"].cpu().numpy(), kw["cu_seqlens_k"].cpu().numpy()
+        eo, el = ref.forward_packed(f64(q), f64(k), f64(v), cq, ck, 1.0, *w)
+        lse = torch.tensor(el, dtype=torch.float32)            # HT [H, T]
+    else:
+        eo, el = ref.forward(f64(q), f64(k), f64(v), 1.0, *w)
+        lse = torch.tensor(el, dtype=torch.float32)[None, None]
+    o = torch.tensor(eo, dtype=torch.float32).to(q.dtype)
+    if not packed:
+        q, k, v, do, o = (t[None, None] for t in (q, k, v, do, o))
+    dq, dk, dv, _ = B.backward(do.to(dev), q.to(dev), k.to(dev), v.to(dev), o.to(dev),
+                               lse.to(dev), sm_scale=1.0, window=w[:2], bottom_right=w[2], **kw)
+    torch.cuda.synchronize()
+    assert B.device_status(dev) == 0
+    sq_ = (lambda t: t.float().cpu().numpy().reshape(-1, t.shape[-1]))
+    return sq_(dq), sq_(dk), sq_(dv)
+
+
+def _bwd_edge_check(dq, dk, dv, sq, sk, w, sign):
+    lo, hi, cnt = ref.row_extent(sq, sk, *w)
+    edge = hi if sign > 0 else lo
+    want = _bwd_edge_expect(sq, sk, edge, cnt)
+    got = dv[:, :8].astype(np.float64)
+    assert np.abs(got - np.rint(got)).max(initial=0) < 1e-3
+    assert np.array_equal(np.rint(got), want), "dV edge counts differ"
+    assert np.abs(dq).max(initial=0) <= 1e-3 and np.abs(dk).max(initial=0) <= 1e-3
+    seen = ref.allowed(sq, sk, *w).any(axis=0)
+    assert np.all(dk[~seen] == 0) and np.all(dv[~seen] == 0), "unseen keys must get 0"
+
+
+@pytest.mark.parametrize("w", WINDOWS, ids=str)
+@pytest.mark.parametrize("sq,sk", SIZES, ids=str)
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16], ids=["bf16", "fp16"])
+def test_backward_edge_probe_dense(dtype, D, sq, sk, w):
+    B = binding()
+    dev = torch.device("cuda")
+    lo, hi, cnt = ref.row_extent(sq, sk, *w)
+    for sign, edge in ((1.0, hi), (-1.0, lo)):
+        q, k, v, do = _bwd_edge_inputs(sq, sk, D, dtype, edge, sign)
+        dq, dk, dv = _bwd_edge_run(B, q, k, v, do, w, dev)
+        _bwd_edge_check(dq, dk, dv, sq, sk, w, sign)
+
+
+@pytest.mark.parametrize("w", WINDOWS, ids=str)
+def test_backward_edge_probe_packed(w):
+    B = binding()
+    dev = torch.device("cuda")
+    from scaled_dot_product_12_b200 import synth
+    sq = [3, 400, 129, 1000, 1, 0]
+    sk = [700, 300, 129, 1100, 64, 5]
+    cu_q, cu_k = synth.cumsum0(sq), synth.cumsum0(sk)
+    for sign in (1.0, -1.0):
+        parts = []
+        for a, b in zip(sq, sk):
+            lo, hi, _ = ref.row_extent(a, b, *w)
+            parts.append(_bwd_edge_inputs(a, b, 64, torch.bfloat16, hi if sign > 0 else lo, sign))
+        q, k, v, do = (torch.cat([p[n] for p in parts])[:, None] for n in range(4))
+        dq, dk, dv = _bwd_edge_run(B, q, k, v, do, w, dev, cu_seqlens_q=cu_q.to(dev),
+                                   cu_seqlens_k=cu_k.to(dev), max_seqlen_q=max(sq),
+                                   max_seqlen_k=max(sk))
+        for s in range(len(sq)):
+            rq = slice(int(cu_q[s]), int(cu_q[s + 1]))
+            rk = slice(int(cu_k[s]), int(cu_k[s + 1]))
+            _bwd_edge_check(dq[rq], dk[rk], dv[rk], sq[s], sk[s], w, sign)

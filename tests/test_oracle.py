@@ -392,3 +392,72 @@ def test_row_subset_equals_full_rows():
     o2, lse2 = ref.forward(q, k, v, 0.4, 50, 3, True, rows=rows)
     np.testing.assert_array_equal(o2, o[rows])
     np.testing.assert_array_equal(lse2, lse[rows])
+
+
+# ---------------------------------------------------------------------------
+# The dense BHSD wrappers: every (b, h) slice is the independent brute force of
+# that slice's own inputs, and a wrapper that mixes up batch and head indices
+# (planted below) fails the same check.
+# ---------------------------------------------------------------------------
+
+def _check_dense_wrappers(fwd_dense, bwd_dense, w):
+    B_, H, sq, sk, d = 2, 3, 6, 9, 4
+    q, k, v, do = (_rand(s, 40 + i) for i, s in
+                   enumerate([(B_, H, sq, d), (B_, H, sk, d), (B_, H, sk, d), (B_, H, sq, d)]))
+    c = 0.45
+    o, lse = fwd_dense(q, k, v, c, *w)
+    dq, dk, dv = bwd_dense(q, k, v, do, c, *w)
+    assert o.shape == q.shape and lse.shape == (B_, H, sq)
+    for b in range(B_):
+        for h in range(H):
+            bo, blse, bdq, bdk, bdv = _brute(q[b, h], k[b, h], v[b, h], do[b, h], c, w)
+            np.testing.assert_allclose(o[b, h], bo, rtol=1e-12, atol=1e-12)
+            np.testing.assert_array_equal(np.isneginf(lse[b, h]), np.isneginf(blse))
+            fin = np.isfinite(blse)
+            np.testing.assert_allclose(lse[b, h][fin], blse[fin], rtol=1e-12, atol=1e-12)
+            for a, e in ((dq[b, h], bdq), (dk[b, h], bdk), (dv[b, h], bdv)):
+                np.testing.assert_allclose(a, e, rtol=1e-10, atol=1e-12)
+    # a subset of heads: those computed, the rest left NaN
+    sub = [(1, 2), (0, 0)]
+    o2, lse2 = fwd_dense(q, k, v, c, *w, heads=sub)
+    g2 = bwd_dense(q, k, v, do, c, *w, heads=sub)
+    for b in range(B_):
+        for h in range(H):
+            if (b, h) in sub:
+                np.testing.assert_array_equal(o2[b, h], o[b, h])
+                for a, e in zip(g2, (dq, dk, dv)):
+                    np.testing.assert_array_equal(a[b, h], e[b, h])
+            else:
+                assert np.isnan(o2[b, h]).all() and np.isnan(lse2[b, h]).all()
+                assert all(np.isnan(a[b, h]).all() for a in g2)
+
+
+@pytest.mark.parametrize("w", [(INF, INF, False), (CTL, 0, False), (2, -1, True), (CBR, 0, True)])
+def test_dense_wrappers_equal_the_brute_force_per_head(w):
+    _check_dense_wrappers(ref.forward_dense, ref.backward_dense, w)
+
+
+def _planted_forward_dense_wrong_head(q, k, v, c, wl, wr, br=False, heads=None):
+    B_, H = q.shape[:2]
+    o, lse = ref.forward_dense(q, k, v, c, wl, wr, br, heads=heads)
+    for b, h in heads if heads is not None else [(b, h) for b in range(B_) for h in range(H)]:
+        # K of the neighbouring head
+        o[b, h], lse[b, h] = ref.forward(q[b, h], k[b, (h + 1) % H], v[b, h], c, wl, wr, br)
+    return o, lse
+
+
+def _planted_backward_dense_batch_swap(q, k, v, do, c, wl, wr, br=False, heads=None):
+    B_, H = q.shape[:2]
+    dq, dk, dv = ref.backward_dense(q, k, v, do, c, wl, wr, br, heads=heads)
+    for b, h in heads if heads is not None else [(b, h) for b in range(B_) for h in range(H)]:
+        # dK stored into the other batch's slot
+        dk[(b + 1) % B_, h] = ref.backward(q[b, h], k[b, h], v[b, h], do[b, h], c, wl, wr, br)[1]
+    return dq, dk, dv
+
+
+def test_planted_dense_wrapper_index_slips_are_caught():
+    w = (INF, INF, False)
+    with pytest.raises(AssertionError):
+        _check_dense_wrappers(_planted_forward_dense_wrong_head, ref.backward_dense, w)
+    with pytest.raises(AssertionError):
+        _check_dense_wrappers(ref.forward_dense, _planted_backward_dense_batch_swap, w)
