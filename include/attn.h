@@ -44,8 +44,13 @@
  *     (rows_q = B*Sq, or total_q for a packed Q side) of 2^31 - 256 or more.  ATTN_ERROR_NO_KERNEL_IMAGE
  *     (cudaErrorNoKernelImageForDevice) on a GPU other than sm_100.  Launch
  *     errors are passed through.  A failing call writes nothing.
- *   - Tensors: fp16 or bf16 (ATTN_DTYPE_*), the head dimension D contiguous
- *     (stride 1), D a multiple of 16 in [16, 128].  Strides are in ELEMENTS.
+ *   - Tensors: fp16 or bf16 (ATTN_DTYPE_*), the head dimension contiguous
+ *     (stride 1), any D in [1, 128]; V, O, dO and dV may have a head
+ *     dimension Dv of their own (version 2; AOTriton 0.15b release notes,
+ *     "Kernel Bug Fixes", name Hdim_vo apart from Hdim_qk).  Strides are in ELEMENTS, and every
+ *     stride's byte size must be a multiple of 16: a D that is not a multiple
+ *     of 8 lives in rows the caller pads (e.g. a [..., 72] buffer viewed as
+ *     [..., 67]); columns past D are never read into a result or written.
  *       dense  (BHSD):  element (b, h, s, d) at base + b*stride[0] + h*stride[1]
  *                       + s*stride[2] + d
  *       packed (1THD):  element (t, h, d) at base + t*stride[2] + h*stride[1] + d
@@ -76,7 +81,11 @@ extern "C" {
 #define ATTN_API
 #endif
 
-#define ATTN_PARAMS_VERSION 1u
+/* Version 2 adds the fields after cu_seqlens_k (forward) / main_kernel_events
+ * (backward).  A caller built against version 1 passes version 1 and the
+ * version-1 struct size (ATTN_FWD_PARAMS_V1_SIZE / ATTN_BWD_PARAMS_V1_SIZE);
+ * the version-2 fields then read as zero. */
+#define ATTN_PARAMS_VERSION 2u
 
 /* Return codes (numeric values of cudaError_t). */
 #define ATTN_SUCCESS 0
@@ -103,7 +112,7 @@ extern "C" {
  * VarlenMode (one byte): bit 0 stacked (0 = BHSD, 1 = 1THD), bits 2:1 length
  * (0 uniform, 1 cumulative sums, 2 per-sequence array), bits 4:3 position
  * (0 uniform, 1 reuse the cumulative sums, 2 second array), bits 7:5
- * reserved.  Each side takes one of three modes on its own (the Q side
+ * reserved.  Each side takes one of five modes on its own (the Q side
  * addresses Q, O, LSE, dO and dQ; the K side K, V, dK and dV):
  *   ATTN_VARLEN_MODE_DENSE   BHSD, every batch Sq queries / Sk keys;
  *   ATTN_VARLEN_MODE_PACKED  1THD, that side's cu_seqlens array holds B + 1
@@ -111,17 +120,31 @@ extern "C" {
  *   ATTN_VARLEN_MODE_PADDED  BHSD sized [B, H, Sq, D] / [B, H, Sk, D], with
  *                            per-batch lengths: that side's cu_seqlens array
  *                            holds B lengths (not cumulative; clamped to
- *                            [0, Sq] / [0, Sk]); rows past a batch's lengths
- *                            are padding: never written, and their contents
- *                            (NaN included) do not reach any result.
- * A batch index b names the same sequence on both sides.
- * Any other mode returns ATTN_ERROR_INVALID_VALUE.
+ *                            [0, Sq] / [0, Sk]);
+ *   ATTN_VARLEN_MODE_PACKED_USED (version 2)
+ *                            1THD whose sequence b occupies rows
+ *                            [cu_seqlens[b], cu_seqlens[b + 1]) (B + 1
+ *                            cumulative entries, the positions) of which the
+ *                            first seqused[b] are used (a packed cache whose
+ *                            slots are longer than their contents);
+ *   ATTN_VARLEN_MODE_PACKED_OFFSETS (version 2)
+ *                            1THD whose sequence b starts at row
+ *                            cu_seqlens[b] (B entries: a second array of
+ *                            positions, in any order) and has seqused[b]
+ *                            rows; the used ranges must not overlap.
+ * In every mode with lengths, rows of a tensor that lie outside every used
+ * range are padding: never written, and their contents (NaN included) do not
+ * reach any result.  Lengths and positions are clamped on the device to the
+ * tensor (and, for PACKED_USED, to the slot).  A batch index b names the same
+ * sequence on both sides.  Any other mode returns ATTN_ERROR_INVALID_VALUE.
  */
 #define ATTN_VARLEN_MODE(stacked, length, position) \
   ((uint32_t)(stacked) | ((uint32_t)(length) << 1) | ((uint32_t)(position) << 3))
 #define ATTN_VARLEN_MODE_DENSE ATTN_VARLEN_MODE(0, 0, 0)
 #define ATTN_VARLEN_MODE_PACKED ATTN_VARLEN_MODE(1, 1, 1)
 #define ATTN_VARLEN_MODE_PADDED ATTN_VARLEN_MODE(0, 2, 0)
+#define ATTN_VARLEN_MODE_PACKED_USED ATTN_VARLEN_MODE(1, 2, 1)
+#define ATTN_VARLEN_MODE_PACKED_OFFSETS ATTN_VARLEN_MODE(1, 2, 2)
 #define ATTN_LSE_HT 0u
 #define ATTN_LSE_TH 1u
 #define ATTN_DIAGONAL_TOP_LEFT 0u
@@ -133,11 +156,27 @@ extern "C" {
 /*
  * Forward parameters.  Sizes: dense -- B batches of Sq queries and Sk keys;
  * packed -- B sequences, Sq / Sk the largest seqlen_q / seqlen_k (they size
- * the launch; a sequence longer than them is an error of the caller),
- * total_q / total_k the rows of the packed tensors, cu_seqlens_q / _k device
- * arrays of B + 1 int32 cumulative lengths starting at 0; padded -- dense
- * tensors of B batches with Sq / Sk rows, cu_seqlens_q / _k device arrays of
- * B int32 lengths (seqlen_q / seqlen_k of each batch).
+ * the launch; a sequence longer than them is an error of the caller, whose
+ * rows past Sq / Sk are left unwritten), total_q / total_k the rows of the
+ * packed tensors, cu_seqlens_q / _k device arrays of B + 1 int32 cumulative
+ * lengths starting at 0 (each entry is clamped to [0, total_q] / [0,
+ * total_k] on the device, so an array that runs past the tensors shortens
+ * the sequences concerned; nothing outside the tensors is read or written);
+ * padded -- dense tensors of B batches with Sq / Sk rows, cu_seqlens_q / _k
+ * device arrays of B int32 lengths (seqlen_q / seqlen_k of each batch);
+ * PACKED_USED / PACKED_OFFSETS -- as packed, with the positions in
+ * cu_seqlens_q / _k and the lengths in seqused_q / _k (see VarlenBits).
+ *
+ * Dropout (version 2; AOTriton 0.10b release notes, "Major Changes from
+ * Release 0.9 Beta": Philox with 32-bit words in groups of four; 0.14b notes,
+ * "Minor Changes from Release 0.13 Beta": the four words of a counter in
+ * generation order): with 0 < dropout_p < 1, element (i, j) of P (query row
+ * i and key j counted within their sequence, head index bh = b * H + h) is
+ * kept iff word (j mod 4) of Philox4x32-10 on the counter
+ * (j div 4, i, bh, philox_offset) under the key (low, high 32 bits of
+ * philox_seed) is below floor((1 - dropout_p) * 2^32); kept elements are
+ * scaled by 1 / (1 - dropout_p).  LSE is that of the softmax without
+ * dropout.  The backward regenerates the same mask from the same fields.
  */
 typedef struct attn_fwd_params {
   uint32_t struct_size; /* sizeof(attn_fwd_params) */
@@ -156,7 +195,16 @@ typedef struct attn_fwd_params {
   uint32_t varlen_bits;
   const int32_t* cu_seqlens_q; /* packed / padded only, device memory */
   const int32_t* cu_seqlens_k;
+  /* ---- version 2 ---- */
+  const int32_t* seqused_q;    /* PACKED_USED / PACKED_OFFSETS: B lengths, device memory */
+  const int32_t* seqused_k;
+  int32_t Dv;                  /* head dim of V and O, in [1, 128]; 0 = D */
+  float dropout_p;             /* [0, 1); 0 = no dropout */
+  uint64_t philox_seed;
+  uint32_t philox_offset;
+  uint32_t flags;              /* none defined for the forward: must be 0 */
 } attn_fwd_params;
+#define ATTN_FWD_PARAMS_V1_SIZE ((uint32_t)offsetof(attn_fwd_params, seqused_q))
 
 /*
  * Backward parameters: the forward's fields plus the forward output O, its
@@ -165,7 +213,8 @@ typedef struct attn_fwd_params {
  * a caller-owned device workspace of attn_bwd_workspace_size() bytes,
  * 256-byte aligned.  The workspace holds, after the call, the fp32 rowsums
  * delta = rowsum(dO o O) [H][rows] followed by the fp32 dQ accumulator
- * [H][rows][D], rows = B*Sq (dense) or total_q (packed).
+ * [H][rows][D], rows = B*Sq (dense) or total_q (packed), and with
+ * ATTN_BWD_DETERMINISTIC the int32 order counters [H][rows][4].
  */
 typedef struct attn_bwd_params {
   uint32_t struct_size; /* sizeof(attn_bwd_params) */
@@ -195,7 +244,22 @@ typedef struct attn_bwd_params {
    * stream's device, recorded on `stream` immediately before and after the
    * main backward kernel (so the caller can time it alone).  NULL: none. */
   void* main_kernel_events[2];
+  /* ---- version 2 ---- */
+  const int32_t* seqused_q;
+  const int32_t* seqused_k;
+  int32_t Dv;                  /* head dim of V, O, dO and dV; 0 = D */
+  float dropout_p;             /* the forward's dropout fields */
+  uint64_t philox_seed;
+  uint32_t philox_offset;
+  uint32_t flags;              /* ATTN_BWD_DETERMINISTIC or 0 */
 } attn_bwd_params;
+#define ATTN_BWD_PARAMS_V1_SIZE ((uint32_t)offsetof(attn_bwd_params, seqused_q))
+
+/* attn_bwd_params.flags: add the dQ contributions of the key tiles in a
+ * fixed order, so that repeated calls give bit-identical dQ (AOTriton 0.15b
+ * release notes, "Known Problems", record run-to-run differences of the
+ * backward).  Costs some speed and H * rows * 16 bytes more workspace. */
+#define ATTN_BWD_DETERMINISTIC 1u
 
 /* Forward: writes O and (unless lse is NULL) LSE.  One kernel launch. */
 ATTN_API int attn_fwd(const attn_fwd_params* params, void* stream);
@@ -224,8 +288,10 @@ ATTN_API size_t attn_bwd_workspace_size(const attn_bwd_params* params);
  *   - Sizes whose attn_bwd_workspace_size() exceeds ATTN_STATIC_WORKSPACE_BYTES
  *     are rejected with cudaErrorMemoryAllocation (2) before any GPU work;
  *     otherwise the return codes are those of attn_bwd.
- *   - The first call on a device looks up that device's address of the array
- *     (once per device); make that first call before any stream capture.
+ *   - Every call looks up the device address of the array on the stream's
+ *     device (so a reset of the device's context, which can move it, is
+ *     harmless); the first call on a device may also load the library's
+ *     device code there, so make that first call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents
  *     there; each call clears the accumulator it needs before use.  Calls whose
  *     work overlaps on the GPU (different streams without ordering between
@@ -260,7 +326,11 @@ ATTN_API int attn_tile_plan_bwd(int32_t seqlen_q, int32_t seqlen_k, int32_t wind
 
 /* Reads and clears the device status word of the stream's device (waits for
  * the stream).  *status = 0 when every device-side wait finished in time;
- * otherwise bit k marks wait site k that gave up.  Returns a cudaError_t. */
+ * otherwise bit k marks wait site k that gave up.  Returns a cudaError_t.
+ * There is one status word per device, shared by every caller and stream on
+ * that device: a bit set by one caller's kernel is seen (and cleared) by
+ * whichever caller reads it first, so callers that run concurrently on one
+ * device and need to attribute a failure must order their reads. */
 ATTN_API int attn_device_status(void* stream, uint32_t* status);
 
 #ifdef __cplusplus

@@ -19,7 +19,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libattn.so")
 
 # Constants of include/attn.h
-PARAMS_VERSION = 1
+PARAMS_VERSION = 2
+BWD_DETERMINISTIC = 1
 DTYPE_FP16, DTYPE_BF16 = 0, 1
 WINDOW_INF = 2**31 - 1
 CAUSAL_TOP_LEFT = -(2**31)
@@ -39,6 +40,8 @@ def varlen_mode(stacked: int, length: int, position: int) -> int:
 MODE_DENSE = varlen_mode(0, 0, 0)
 MODE_PACKED = varlen_mode(1, 1, 1)
 MODE_PADDED = varlen_mode(0, 2, 0)
+MODE_PACKED_USED = varlen_mode(1, 2, 1)
+MODE_PACKED_OFFSETS = varlen_mode(1, 2, 2)
 
 
 def varlen_bits(qmode: int, kmode: int, lse_layout: int, diagonal: int) -> int:
@@ -59,6 +62,10 @@ class FwdParams(ctypes.Structure):
         ("sm_scale", ctypes.c_float), ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32), ("varlen_bits", ctypes.c_uint32),
         ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        # version 2
+        ("seqused_q", ctypes.c_void_p), ("seqused_k", ctypes.c_void_p), ("Dv", ctypes.c_int32),
+        ("dropout_p", ctypes.c_float), ("philox_seed", ctypes.c_uint64),
+        ("philox_offset", ctypes.c_uint32), ("flags", ctypes.c_uint32),
     ]
 
 
@@ -77,7 +84,16 @@ class BwdParams(ctypes.Structure):
         ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("main_kernel_events", ctypes.c_void_p * 2),
+        # version 2
+        ("seqused_q", ctypes.c_void_p), ("seqused_k", ctypes.c_void_p), ("Dv", ctypes.c_int32),
+        ("dropout_p", ctypes.c_float), ("philox_seed", ctypes.c_uint64),
+        ("philox_offset", ctypes.c_uint32), ("flags", ctypes.c_uint32),
     ]
+
+
+# Size of the version-1 structs (every field before seqused_q).
+FWD_PARAMS_V1_SIZE = FwdParams.seqused_q.offset
+BWD_PARAMS_V1_SIZE = BwdParams.seqused_q.offset
 
 
 EXPORTS = {
@@ -154,29 +170,51 @@ def _stream_handle(device: torch.device, stream) -> int:
 
 
 class Problem:
-    """Sizes, window and layout of one call, shared by forward and backward."""
+    """Sizes, window and layout of one call, shared by forward and backward.
+
+    Each side on its own: dense (4-D [B, H, S, D]), padded (4-D with
+    ``seqlens``: B lengths), packed (3-D [T, H, D] with ``cu_seqlens``: B + 1
+    cumulative lengths), packed with used lengths (``cu_seqlens`` as slots
+    plus ``seqused``: B lengths) or packed at positions (``seqstart``: B
+    start rows plus ``seqused``).
+    """
 
     def __init__(self, q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
-                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q=None, seqlens_k=None):
-        # Each side on its own: packed (cu_seqlens, 3-D [T, H, D] tensors),
-        # padded (seqlens, 4-D [B, H, S, D] tensors) or dense (4-D).
-        if cu_seqlens_q is not None and seqlens_q is not None or \
-                cu_seqlens_k is not None and seqlens_k is not None:
-            raise ValueError("a side is packed (cu_seqlens) or padded (seqlens), not both")
-        self.q_packed, self.k_packed = cu_seqlens_q is not None, cu_seqlens_k is not None
-        self.q_padded, self.k_padded = seqlens_q is not None, seqlens_k is not None
+                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q=None, seqlens_k=None,
+                 seqused_q=None, seqused_k=None, seqstart_q=None, seqstart_k=None):
+        sides = {}
+        for name, cu, lens, used, start in (("q", cu_seqlens_q, seqlens_q, seqused_q, seqstart_q),
+                                            ("k", cu_seqlens_k, seqlens_k, seqused_k, seqstart_k)):
+            given = [x is not None for x in (cu, lens, start)]
+            if sum(given) > 1:
+                raise ValueError(f"{name}: give one of cu_seqlens, seqlens or seqstart")
+            if used is not None and cu is None and start is None:
+                raise ValueError(f"{name}: seqused needs cu_seqlens (slots) or seqstart (positions)")
+            if start is not None and used is None:
+                raise ValueError(f"{name}: seqstart needs seqused")
+            if cu is not None:
+                mode = MODE_PACKED_USED if used is not None else MODE_PACKED
+                count, ptr = cu.numel() - 1, cu
+            elif start is not None:
+                mode, count, ptr = MODE_PACKED_OFFSETS, start.numel(), start
+            elif lens is not None:
+                mode, count, ptr = MODE_PADDED, lens.numel(), lens
+            else:
+                mode, count, ptr = MODE_DENSE, None, None
+            if used is not None and used.numel() != count:
+                raise ValueError(f"{name}: seqused needs one entry per sequence")
+            sides[name] = (mode, count, ptr, used)
+        (qmode, qcount, self.cu_q, self.used_q) = sides["q"]
+        (kmode, kcount, self.cu_k, self.used_k) = sides["k"]
+        self.q_packed, self.k_packed = bool(qmode & 1), bool(kmode & 1)
+        self.q_padded, self.k_padded = qmode == MODE_PADDED, kmode == MODE_PADDED
         for name, packed, t in (("q", self.q_packed, q), ("k", self.k_packed, k)):
             if t.dim() != (3 if packed else 4):
                 raise ValueError(f"{name}: packed inputs are [tokens, H, D], others [B, H, S, D]")
         sizes = set()
-        if self.q_packed:
-            sizes.add(cu_seqlens_q.numel() - 1)
-        elif self.q_padded:
-            sizes.add(seqlens_q.numel())
-        if self.k_packed:
-            sizes.add(cu_seqlens_k.numel() - 1)
-        elif self.k_padded:
-            sizes.add(seqlens_k.numel())
+        for count in (qcount, kcount):
+            if count is not None:
+                sizes.add(count)
         if not self.q_packed:
             sizes.add(q.shape[0])
         if not self.k_packed:
@@ -195,18 +233,18 @@ class Problem:
         self.window = (int(window[0]), int(window[1]))
         self.bottom_right = bool(bottom_right)
         self.lse_th = (lse_layout.upper() == "TH")
-        qmode = MODE_PACKED if self.q_packed else (MODE_PADDED if self.q_padded else MODE_DENSE)
-        kmode = MODE_PACKED if self.k_packed else (MODE_PADDED if self.k_padded else MODE_DENSE)
         self.bits = varlen_bits(qmode, kmode, LSE_TH if self.lse_th else LSE_HT,
                                 DIAGONAL_BOTTOM_RIGHT if self.bottom_right else DIAGONAL_TOP_LEFT)
-        # the pointer fields carry whichever array each side's mode names
-        self.cu_q = cu_seqlens_q if self.q_packed else seqlens_q
-        self.cu_k = cu_seqlens_k if self.k_packed else seqlens_k
+        self.dropout_p, self.philox_seed, self.philox_offset = 0.0, 0, 0
+        self.flags = 0
 
     def lse_shape(self):
         if self.q_packed:
             return (self.total_q, self.H) if self.lse_th else (self.H, self.total_q)
         return (self.B, self.Sq, self.H) if self.lse_th else (self.B, self.H, self.Sq)
+
+    def set_dropout(self, p, seed, offset):
+        self.dropout_p, self.philox_seed, self.philox_offset = float(p), int(seed), int(offset)
 
     def fill(self, p, dtype_code):
         p.struct_size = ctypes.sizeof(p)
@@ -219,21 +257,34 @@ class Problem:
         p.varlen_bits = self.bits
         p.cu_seqlens_q = _ptr(self.cu_q)
         p.cu_seqlens_k = _ptr(self.cu_k)
+        p.seqused_q = _ptr(self.used_q)
+        p.seqused_k = _ptr(self.used_k)
+        p.dropout_p = self.dropout_p
+        p.philox_seed = self.philox_seed & (2**64 - 1)
+        p.philox_offset = self.philox_offset & 0xFFFFFFFF
+        p.flags = self.flags
 
 
 def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_right=False,
             cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None,
             lse_layout="HT", out=None, lse=None, return_lse=True, stream=None,
-            seqlens_q=None, seqlens_k=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            seqlens_q=None, seqlens_k=None, seqused_q=None, seqused_k=None, seqstart_q=None,
+            seqstart_k=None, dropout_p=0.0, philox_seed=0,
+            philox_offset=0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """O (and LSE) of FlashAttention through attn_fwd.
 
     Dense: q [B,H,Sq,D], k/v [B,H,Sk,D].  Packed: q [Tq,H,D], k/v [Tk,H,D] with
-    int32 cu_seqlens on the device and the largest sequence lengths.  Padded:
-    dense shapes plus int32 seqlens_q / seqlens_k [B] on the device; rows past
-    a batch's lengths are left untouched.
+    int32 cu_seqlens on the device and the largest sequence lengths; with
+    seqused as well, sequence b uses the first seqused[b] rows of its slot;
+    seqstart (B start rows) with seqused places the sequences anywhere in the
+    packed tensor.  Padded: dense shapes plus int32 seqlens_q / seqlens_k [B]
+    on the device.  Rows outside every sequence are left untouched.  dropout_p
+    > 0 drops elements of P with the Philox generator keyed by philox_seed.
     """
     pr = Problem(q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
-                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k)
+                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k, seqused_q,
+                 seqused_k, seqstart_q, seqstart_k)
+    pr.set_dropout(dropout_p, philox_seed, philox_offset)
     if out is None:
         out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
     if lse is None and return_lse:
@@ -241,6 +292,7 @@ def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_righ
     p = FwdParams()
     pr.fill(p, _dtype_code(q))
     p.q, p.k, p.v, p.o, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse)
+    p.Dv = v.shape[-1]
     p.q_stride = _strides(q, pr.q_packed)
     p.k_stride = _strides(k, pr.k_packed)
     p.v_stride = _strides(v, pr.k_packed)
@@ -254,6 +306,7 @@ def bwd_params(dout, q, k, v, o, lse, pr: Problem, dq, dk, dv, workspace=None) -
     pr.fill(p, _dtype_code(q))
     p.q, p.k, p.v, p.o, p.dout, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse)
     p.dq, p.dk, p.dv = _ptr(dq), _ptr(dk), _ptr(dv)
+    p.Dv = v.shape[-1]
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", dout), ("dq", dq), ("dk", dk),
                     ("dv", dv)):
         setattr(p, name + "_stride", _strides(t, pr.k_packed if name in ("k", "v", "dk", "dv")
@@ -271,10 +324,16 @@ def workspace_bytes(p: BwdParams) -> int:
 def backward(dout, q, k, v, o, lse, sm_scale=None, window=(WINDOW_INF, WINDOW_INF),
              bottom_right=False, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
              max_seqlen_k=None, lse_layout="HT", dq=None, dk=None, dv=None, workspace=None,
-             stream=None, seqlens_q=None, seqlens_k=None):
-    """(dQ, dK, dV) through attn_bwd; the workspace is allocated if not given."""
+             stream=None, seqlens_q=None, seqlens_k=None, seqused_q=None, seqused_k=None,
+             seqstart_q=None, seqstart_k=None, dropout_p=0.0, philox_seed=0, philox_offset=0,
+             deterministic=False):
+    """(dQ, dK, dV) through attn_bwd; the workspace is allocated if not given.
+    ``deterministic`` adds the dQ contributions in a fixed order."""
     pr = Problem(q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
-                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k)
+                 max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k, seqused_q,
+                 seqused_k, seqstart_q, seqstart_k)
+    pr.set_dropout(dropout_p, philox_seed, philox_offset)
+    pr.flags = BWD_DETERMINISTIC if deterministic else 0
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

@@ -43,11 +43,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Per-device facts, filled once under a lock: is it sm_100, and where is its
-// copy of the status word.
+// Per-device facts that outlive a context reset (compute capability, SM
+// count), filled once under a lock.  The status word's device address is not
+// cached: a reset of the device's primary context can move it, so every call
+// looks it up (cheap once the module is loaded).
 struct DeviceInfo {
   bool ready = false;
   bool sm100 = false;
+  int sms = 0;
   uint32_t* status = nullptr;
 };
 std::mutex g_dev_mu;
@@ -55,25 +58,31 @@ DeviceInfo g_dev[kMaxDevices];
 
 cudaError_t device_info(int dev, DeviceInfo* out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
-    int major = 0, minor = 0;
-    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    if (e != cudaSuccess) return e;
-    d.sm100 = (major == 10 && minor == 0);
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_status);  // current device == dev here
-    if (e != cudaSuccess) return e;
-    d.status = static_cast<uint32_t*>(p);
-    d.ready = true;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+      int major = 0, minor = 0, sms = 0;
+      cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      d.sm100 = (major == 10 && minor == 0);
+      d.sms = sms;
+      d.ready = true;
+    }
+    *out = d;
   }
-  *out = d;
+  if (!out->sm100) return cudaSuccess;
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_status);  // current device == dev here
+  if (e != cudaSuccess) return e;
+  out->status = static_cast<uint32_t*>(p);
   return cudaSuccess;
 }
 
-// Runs `fn` with the stream's device current, restoring the caller's device.
+// Runs `fn` with the stream's device current, restoring the caller's device;
+// a failure to restore it is reported when the call itself succeeded.
 template <class F>
 cudaError_t on_stream_device(cudaStream_t stream, F&& fn) {
   int cur = 0, dev = 0;
@@ -87,8 +96,11 @@ cudaError_t on_stream_device(cudaStream_t stream, F&& fn) {
   if (dev != cur && (e = cudaSetDevice(dev)) != cudaSuccess) return e;
   DeviceInfo info;
   e = device_info(dev, &info);
-  if (e == cudaSuccess) e = info.sm100 ? fn(info) : cudaErrorNoKernelImageForDevice;
-  if (dev != cur) cudaSetDevice(cur);
+  if (e == cudaSuccess) e = info.sm100 ? fn(dev, info) : cudaErrorNoKernelImageForDevice;
+  if (dev != cur) {
+    const cudaError_t r = cudaSetDevice(cur);
+    if (e == cudaSuccess) e = r;
+  }
   return e;
 }
 
@@ -97,8 +109,10 @@ constexpr uint32_t kModeReserved = 0xE0u;        // bits 7:5 of a VarlenMode
 
 // Addressing of each side (Q: Q, O, LSE, dO, dQ; K: K, V, dK, dV).
 struct Mode {
-  bool q_packed, k_packed;  // 1THD with cumulative lengths
-  bool q_padded, k_padded;  // BHSD with per-batch lengths
+  bool q_packed, k_packed;    // 1THD (stacked), positions from cu_seqlens
+  bool q_used, k_used;        // stacked, lengths from seqused
+  bool q_offsets, k_offsets;  // stacked, cu_seqlens holds B start rows (not cumulative)
+  bool q_padded, k_padded;    // BHSD with per-batch lengths
   bool lse_th;
   bool bottom_right;
 };
@@ -108,17 +122,43 @@ bool decode_bits(uint32_t bits, Mode* m) {
   const uint32_t qm = bits & 0xFFu, km = (bits >> 8) & 0xFFu, lse = (bits >> 16) & 3u;
   if ((qm | km) & kModeReserved) return false;
   auto known = [](uint32_t x) {
-    return x == ATTN_VARLEN_MODE_DENSE || x == ATTN_VARLEN_MODE_PACKED || x == ATTN_VARLEN_MODE_PADDED;
+    return x == ATTN_VARLEN_MODE_DENSE || x == ATTN_VARLEN_MODE_PACKED ||
+           x == ATTN_VARLEN_MODE_PADDED || x == ATTN_VARLEN_MODE_PACKED_USED ||
+           x == ATTN_VARLEN_MODE_PACKED_OFFSETS;
   };
-  if (!known(qm) || !known(km)) return false;  // each side on its own: dense, packed or padded
+  if (!known(qm) || !known(km)) return false;  // each side on its own
   if (lse > 1) return false;
-  m->q_packed = (qm == ATTN_VARLEN_MODE_PACKED);
-  m->k_packed = (km == ATTN_VARLEN_MODE_PACKED);
+  auto stacked = [](uint32_t x) { return (x & 1u) != 0; };
+  m->q_packed = stacked(qm);
+  m->k_packed = stacked(km);
+  m->q_used = (qm == ATTN_VARLEN_MODE_PACKED_USED || qm == ATTN_VARLEN_MODE_PACKED_OFFSETS);
+  m->k_used = (km == ATTN_VARLEN_MODE_PACKED_USED || km == ATTN_VARLEN_MODE_PACKED_OFFSETS);
+  m->q_offsets = (qm == ATTN_VARLEN_MODE_PACKED_OFFSETS);
+  m->k_offsets = (km == ATTN_VARLEN_MODE_PACKED_OFFSETS);
   m->q_padded = (qm == ATTN_VARLEN_MODE_PADDED);
   m->k_padded = (km == ATTN_VARLEN_MODE_PADDED);
   m->lse_th = (lse == ATTN_LSE_TH);
   m->bottom_right = ((bits >> 18) & 1u) != 0;
   return true;
+}
+
+// Copies a version-1 or version-2 params struct into a full version-2 one
+// (version-1 callers get zeros in the fields they do not know).
+template <class P>
+bool normalize(const P* in, uint32_t v1_size, P* out) {
+  if (!in) return false;
+  if (in->version == ATTN_PARAMS_VERSION && in->struct_size == sizeof(P)) {
+    std::memcpy(out, in, sizeof(P));
+    return true;
+  }
+  if (in->version == 1u && in->struct_size == v1_size) {
+    std::memset(out, 0, sizeof(P));
+    std::memcpy(out, in, v1_size);
+    out->struct_size = sizeof(P);
+    out->version = ATTN_PARAMS_VERSION;
+    return true;
+  }
+  return false;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -159,14 +199,14 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// 2-D fp32 map over the dQ accumulator [H*rows][D] (row pitch D*4 bytes),
+// 2-D fp32 map over the dQ accumulator [H*rows][D] (row pitch DA*4 bytes),
 // 32 x 32 boxes with 128-byte swizzle: the backward adds staged dQ tiles
 // through it.
-cudaError_t make_dq_map(CUtensorMap* map, float* base, int D, int64_t rows_total) {
+cudaError_t make_dq_map(CUtensorMap* map, float* base, int D, int DA, int64_t rows_total) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(rows_total > 0 ? rows_total : 1)};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+  cuuint64_t strides[1] = {(cuuint64_t)DA * 4};
   cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
@@ -175,35 +215,58 @@ cudaError_t make_dq_map(CUtensorMap* map, float* base, int D, int64_t rows_total
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Checks shared by forward and backward.
+// Checks shared by forward and backward (on a normalized struct).
 template <class P>
-bool common_ok(const P* p, size_t want_size, Mode* m, bool check_pointers = true) {
-  if (!p || p->struct_size != want_size || p->version != ATTN_PARAMS_VERSION) return false;
+bool common_ok(const P* p, Mode* m, uint32_t known_flags, bool check_pointers = true,
+               bool dropout_built = true) {
   if (p->dtype != ATTN_DTYPE_FP16 && p->dtype != ATTN_DTYPE_BF16) return false;
-  if (p->D < 16 || p->D > 128 || (p->D % 16) != 0) return false;
+  if (p->D < 1 || p->D > 128) return false;
   if (p->B < 0 || p->H < 0 || p->Sq < 0 || p->Sk < 0) return false;
   if (p->Sq >= attn::kBig || p->Sk >= attn::kBig) return false;
   if (!std::isfinite(p->sm_scale)) return false;
   if (!decode_bits(p->varlen_bits, m)) return false;
   if (m->q_packed && (p->total_q < 0 || p->total_q >= attn::kBig)) return false;
   if (m->k_packed && (p->total_k < 0 || p->total_k >= attn::kBig)) return false;
-  // Packed and padded sides read their lengths from the device arrays.
+  if ((p->flags & ~known_flags) != 0) return false;
+  if (p->Dv < 0 || p->Dv > 128) return false;  // 0: V and O share D
+  if (!(p->dropout_p >= 0.f && p->dropout_p < 1.f)) return false;  // NaN fails too
+  if (p->dropout_p != 0.f && !dropout_built) return false;
+  // Stacked and padded sides read their positions / lengths from the device
+  // arrays.
   if (check_pointers && p->B > 0) {
     if ((m->q_packed || m->q_padded) && !p->cu_seqlens_q) return false;
     if ((m->k_packed || m->k_padded) && !p->cu_seqlens_k) return false;
+    if (m->q_used && !p->seqused_q) return false;
+    if (m->k_used && !p->seqused_k) return false;
   }
   return true;
 }
 
 bool has_work(int B, int H, int64_t rows_q) { return B > 0 && H > 0 && rows_q > 0; }
 
+// Dropout fields of the kernel arguments: keep iff the Philox word is below
+// floor((1 - p) 2^32); a p so small that every word is kept is no dropout.
+template <class Args, class P>
+void set_dropout(Args& a, const P* p) {
+  const double keep = std::floor((1.0 - (double)p->dropout_p) * 4294967296.0);
+  a.dropout = p->dropout_p > 0.f && keep < 4294967296.0;
+  a.keep_below = a.dropout ? (uint32_t)keep : 0u;
+  a.drop_scale = a.dropout ? (float)(1.0 / (1.0 - (double)p->dropout_p)) : 1.f;
+  a.seed_lo = (uint32_t)(p->philox_seed & 0xFFFFFFFFu);
+  a.seed_hi = (uint32_t)(p->philox_seed >> 32);
+  a.philox_offset = p->philox_offset;
+}
+
 }  // namespace
 
 extern "C" {
 
-int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
+int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
+  attn_fwd_params full;
+  if (!normalize(params, ATTN_FWD_PARAMS_V1_SIZE, &full)) return cudaErrorInvalidValue;
+  const attn_fwd_params* p = &full;
   Mode m;
-  if (!common_ok(p, sizeof(attn_fwd_params), &m)) return cudaErrorInvalidValue;
+  if (!common_ok(p, &m, /*known_flags=*/0u)) return cudaErrorInvalidValue;
   const int64_t rows_q = m.q_packed ? p->total_q : (int64_t)p->B * p->Sq;
   const int64_t rows_k = m.k_packed ? p->total_k : (int64_t)p->B * p->Sk;
   if (!has_work(p->B, p->H, rows_q)) return cudaSuccess;
@@ -220,14 +283,15 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
     return cudaErrorInvalidValue;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  return on_stream_device(stream, [&](const DeviceInfo& info) -> cudaError_t {
+  return on_stream_device(stream, [&](int dev, const DeviceInfo& info) -> cudaError_t {
     attn::FwdArgs a;
     std::memset(&a, 0, sizeof(a));
     const void* kbase = rows_k > 0 ? p->k : p->q;
     const void* vbase = rows_k > 0 ? p->v : p->q;
+    const int Dv = p->Dv ? p->Dv : p->D;
     cudaError_t e = make_map(&a.tq, p->q, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
     if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
-    if (e == cudaSuccess) e = make_map(&a.tv, vbase, p->D, nk, p->H, p->B, p->v_stride, m.k_packed);
+    if (e == cudaSuccess) e = make_map(&a.tv, vbase, Dv, nk, p->H, p->B, p->v_stride, m.k_packed);
     if (e != cudaSuccess) return e;
     a.o = p->o;
     a.lse = p->lse;
@@ -239,6 +303,9 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
     a.Sq = p->Sq;
     a.Sk = p->Sk;
     a.D = p->D;
+    a.D16 = (p->D + 15) / 16 * 16;
+    a.Dv = Dv;
+    a.Dv16 = (Dv + 15) / 16 * 16;
     a.wl = p->window_left;
     a.wr = p->window_right;
     a.bottom_right = m.bottom_right;
@@ -246,28 +313,61 @@ int attn_fwd(const attn_fwd_params* p, void* stream_ptr) {
     a.k_packed = m.k_packed;
     a.q_padded = m.q_padded;
     a.k_padded = m.k_padded;
+    a.q_used = m.q_used;
+    a.k_used = m.k_used;
+    a.q_offsets = m.q_offsets;
+    a.k_offsets = m.k_offsets;
+    a.used_q = p->seqused_q;
+    a.used_k = p->seqused_k;
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.negate = p->sm_scale < 0.f;
     a.total_q = p->total_q;
+    a.total_k = p->total_k;
     a.scale_log2 = std::fabs(p->sm_scale) * 1.4426950408889634f;
     a.status = info.status;
+    a.dev = dev;
+    a.sms = info.sms;
+    set_dropout(a, p);
     return attn::launch_fwd(a, stream);
   });
 }
 
-size_t attn_bwd_workspace_size(const attn_bwd_params* p) {
-  Mode m;
-  if (!common_ok(p, sizeof(attn_bwd_params), &m, /*check_pointers=*/false)) return 0;
+namespace {
+// Workspace of the backward: delta [H][rows] fp32 (256-byte aligned), the dQ
+// accumulator [H][rows][D] fp32, and with ATTN_BWD_DETERMINISTIC the order
+// counters [H][rows][4] int32.
+struct BwdWorkspace {
+  size_t delta_bytes, acc_bytes, order_bytes;
+  size_t total() const { return delta_bytes + acc_bytes + order_bytes; }
+};
+BwdWorkspace bwd_workspace(const attn_bwd_params* p, const Mode& m) {
   const int64_t rows = m.q_packed ? p->total_q : (int64_t)p->B * p->Sq;
   const int64_t n = (int64_t)p->H * rows;
-  const size_t delta_bytes = ((size_t)n * 4 + 255) & ~(size_t)255;
-  return delta_bytes + (size_t)n * p->D * 4;
+  BwdWorkspace w;
+  w.delta_bytes = ((size_t)n * 4 + 255) & ~(size_t)255;
+  w.acc_bytes = (size_t)n * ((p->D + 7) / 8 * 8) * 4;
+  w.order_bytes = (p->flags & ATTN_BWD_DETERMINISTIC) ? (size_t)n * 16 : 0;
+  return w;
+}
+constexpr uint32_t kBwdFlags = ATTN_BWD_DETERMINISTIC;  // flags the backward accepts
+constexpr bool kBwdDropout = true;                       // backward dropout kernels built
+}  // namespace
+
+size_t attn_bwd_workspace_size(const attn_bwd_params* params) {
+  attn_bwd_params full;
+  if (!normalize(params, ATTN_BWD_PARAMS_V1_SIZE, &full)) return 0;
+  Mode m;
+  if (!common_ok(&full, &m, kBwdFlags, /*check_pointers=*/false, kBwdDropout)) return 0;
+  return bwd_workspace(&full, m).total();
 }
 
-int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
+int attn_bwd(const attn_bwd_params* params, void* stream_ptr) {
+  attn_bwd_params full;
+  if (!normalize(params, ATTN_BWD_PARAMS_V1_SIZE, &full)) return cudaErrorInvalidValue;
+  const attn_bwd_params* p = &full;
   Mode m;
-  if (!common_ok(p, sizeof(attn_bwd_params), &m)) return cudaErrorInvalidValue;
+  if (!common_ok(p, &m, kBwdFlags, true, kBwdDropout)) return cudaErrorInvalidValue;
   const int64_t rows_q = m.q_packed ? p->total_q : (int64_t)p->B * p->Sq;
   const int64_t rows_k = m.k_packed ? p->total_k : (int64_t)p->B * p->Sk;
   if (!has_work(p->B, p->H, rows_q) && !(p->B > 0 && p->H > 0 && rows_k > 0)) return cudaSuccess;
@@ -282,7 +382,8 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
   // The dQ accumulator is reduced into through a 2-D tensor map whose row
   // coordinate (head * rows + row) is a signed 32-bit TMA coordinate.
   if ((int64_t)p->H * rows_q >= ((int64_t)1 << 31) - 256) return cudaErrorInvalidValue;
-  const size_t ws = attn_bwd_workspace_size(p);
+  const BwdWorkspace wl = bwd_workspace(p, m);
+  const size_t ws = wl.total();
   if (ws > 0 && (!p->workspace || p->workspace_bytes < ws ||
                  (reinterpret_cast<uintptr_t>(p->workspace) & 255u)))
     return cudaErrorInvalidValue;
@@ -295,18 +396,19 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     if (!strides_ok(st, m.k_packed, p->B, p->H, nk)) return cudaErrorInvalidValue;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  return on_stream_device(stream, [&](const DeviceInfo& info) -> cudaError_t {
+  return on_stream_device(stream, [&](int dev, const DeviceInfo& info) -> cudaError_t {
     attn::BwdArgs a;
     std::memset(&a, 0, sizeof(a));
     const void* qbase = rows_q > 0 ? p->q : p->k;
     const void* dobase = rows_q > 0 ? p->dout : p->k;
     const void* kbase = rows_k > 0 ? p->k : p->q;
     const void* vbase = rows_k > 0 ? p->v : p->q;
+    const int Dv = p->Dv ? p->Dv : p->D;
     cudaError_t e = make_map(&a.tq, qbase, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
     if (e == cudaSuccess)
-      e = make_map(&a.tdo, dobase, p->D, nq, p->H, p->B, p->do_stride, m.q_packed);
+      e = make_map(&a.tdo, dobase, Dv, nq, p->H, p->B, p->do_stride, m.q_packed);
     if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
-    if (e == cudaSuccess) e = make_map(&a.tv, vbase, p->D, nk, p->H, p->B, p->v_stride, m.k_packed);
+    if (e == cudaSuccess) e = make_map(&a.tv, vbase, Dv, nk, p->H, p->B, p->v_stride, m.k_packed);
     if (e != cudaSuccess) return e;
     a.o = p->o;
     a.dout = p->dout;
@@ -328,6 +430,9 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     a.Sq = p->Sq;
     a.Sk = p->Sk;
     a.D = p->D;
+    a.D16 = (p->D + 15) / 16 * 16;
+    a.Dv = Dv;
+    a.Dv16 = (Dv + 15) / 16 * 16;
     a.wl = p->window_left;
     a.wr = p->window_right;
     a.bottom_right = m.bottom_right;
@@ -335,22 +440,35 @@ int attn_bwd(const attn_bwd_params* p, void* stream_ptr) {
     a.k_packed = m.k_packed;
     a.q_padded = m.q_padded;
     a.k_padded = m.k_padded;
+    a.q_used = m.q_used;
+    a.k_used = m.k_used;
+    a.q_offsets = m.q_offsets;
+    a.k_offsets = m.k_offsets;
+    a.used_q = p->seqused_q;
+    a.used_k = p->seqused_k;
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.total_q = p->total_q;
+    a.total_k = p->total_k;
     a.rows = rows_q;
+    a.DA = (p->D + 7) / 8 * 8;
     a.sm_scale = p->sm_scale;
     // c = sm_scale * log2(e); the kernel subtracts LSE*log2(e)/c inside the
     // S^T product, so |c| is kept at least 2^-100.  Below that c * S^T is far
     // under the rounding of LSE*log2(e) and P is unchanged in fp32.
     a.scale_log2 = p->sm_scale * 1.4426950408889634f;
     if (std::fabs(a.scale_log2) < 0x1p-100f) a.scale_log2 = std::signbit(a.scale_log2) ? -0x1p-100f : 0x1p-100f;
-    const size_t delta_bytes = ((size_t)p->H * rows_q * 4 + 255) & ~(size_t)255;
     a.delta = static_cast<float*>(p->workspace);
-    a.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(p->workspace) + delta_bytes);
-    e = make_dq_map(&a.tdq, a.dq_acc, p->D, (int64_t)p->H * rows_q);
+    a.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(p->workspace) + wl.delta_bytes);
+    a.order = wl.order_bytes ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(p->workspace) +
+                                                          wl.delta_bytes + wl.acc_bytes)
+                             : nullptr;
+    e = make_dq_map(&a.tdq, a.dq_acc, p->D, a.DA, (int64_t)p->H * rows_q);
     if (e != cudaSuccess) return e;
     a.status = info.status;
+    a.dev = dev;
+    a.sms = info.sms;
+    set_dropout(a, p);
     a.main_events[0] = static_cast<cudaEvent_t>(p->main_kernel_events[0]);
     a.main_events[1] = static_cast<cudaEvent_t>(p->main_kernel_events[1]);
     return attn::launch_bwd(a, stream);
@@ -401,7 +519,7 @@ int attn_tile_plan_bwd(int32_t seqlen_q, int32_t seqlen_k, int32_t window_left,
 int attn_device_status(void* stream_ptr, uint32_t* status) {
   if (!status) return cudaErrorInvalidValue;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  return on_stream_device(stream, [&](const DeviceInfo& info) -> cudaError_t {
+  return on_stream_device(stream, [&](int, const DeviceInfo& info) -> cudaError_t {
     uint32_t host = 0;
     cudaError_t e = cudaMemcpyAsync(&host, info.status, 4, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);

@@ -45,33 +45,68 @@ template <bool BF16>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant__ BwdArgs a) {
   const int64_t n_groups = (int64_t)a.H * a.rows;
   const int sub = threadIdx.x & 15;
-  const int chunks = a.D / 8;
+  const int chunks = (a.Dv + 7) / 8;  // of O and dO, 8 columns each; the last may be partial
   for (int64_t g = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4); g < n_groups;
        g += (int64_t)gridDim.x * 16) {
     const int h = (int)(g / a.rows);
     const int64_t row = g % a.rows;
     float acc = 0.f;
     if (sub < chunks) {
-      const uint4 ov = *reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint8_t*>(a.o) +
-          2 * (row_offset(a.o_stride, row, h, a.Sq, a.q_packed) + 8 * sub));
-      const uint4 dv = *reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint8_t*>(a.dout) +
-          2 * (row_offset(a.do_stride, row, h, a.Sq, a.q_packed) + 8 * sub));
-      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+      const uint16_t* orow = reinterpret_cast<const uint16_t*>(a.o) +
+                             row_offset(a.o_stride, row, h, a.Sq, a.q_packed) + 8 * sub;
+      const uint16_t* drow = reinterpret_cast<const uint16_t*>(a.dout) +
+                             row_offset(a.do_stride, row, h, a.Sq, a.q_packed) + 8 * sub;
+      uint32_t ow[4], dw[4];
+      if (8 * sub + 8 <= a.Dv) {
+        const uint4 ov = *reinterpret_cast<const uint4*>(orow);
+        const uint4 dv = *reinterpret_cast<const uint4*>(drow);
+        ow[0] = ov.x, ow[1] = ov.y, ow[2] = ov.z, ow[3] = ov.w;
+        dw[0] = dv.x, dw[1] = dv.y, dw[2] = dv.z, dw[3] = dv.w;
+      } else {  // columns past Dv are not read
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = 8 * sub + 2 * e;
+          const uint32_t o0 = c0 < a.Dv ? orow[2 * e] : 0u, o1 = c0 + 1 < a.Dv ? orow[2 * e + 1] : 0u;
+          const uint32_t d0 = c0 < a.Dv ? drow[2 * e] : 0u, d1 = c0 + 1 < a.Dv ? drow[2 * e + 1] : 0u;
+          ow[e] = o0 | (o1 << 16);
+          dw[e] = d0 | (d1 << 16);
+        }
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 x = unpack2<BF16>(ow[e]), y = unpack2<BF16>(dw[e]);
         acc = fmaf(x.x, y.x, acc);
         acc = fmaf(x.y, y.y, acc);
       }
-      float4* z = reinterpret_cast<float4*>(a.dq_acc + g * a.D + 8 * sub);
+    }
+    if (sub < a.DA / 8) {
+      float4* z = reinterpret_cast<float4*>(a.dq_acc + g * a.DA + 8 * sub);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.order && sub == 0) reinterpret_cast<int4*>(a.order)[g] = make_int4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int m = 8; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
     if (sub == 0) a.delta[g] = acc;
+  }
+}
+
+// Eight fp32 values (u, v) times s as 16-bit values at dst, only the first
+// `ncols` of them (dst is 16-byte aligned when ncols >= 8).
+template <bool BF16>
+__device__ __forceinline__ void store_chunk8(uint8_t* dst, float4 u, float4 v, float s, int ncols) {
+  const uint32_t w[4] = {pack2<BF16>(u.x * s, u.y * s), pack2<BF16>(u.z * s, u.w * s),
+                         pack2<BF16>(v.x * s, v.y * s), pack2<BF16>(v.z * s, v.w * s)};
+  if (ncols >= 8) {
+    st_global_v4(dst, w[0], w[1], w[2], w[3]);
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if (2 * e + 1 < ncols)
+      *reinterpret_cast<uint32_t*>(dst + 4 * e) = w[e];
+    else if (2 * e < ncols)
+      *reinterpret_cast<uint16_t*>(dst + 4 * e) = (uint16_t)(w[e] & 0xFFFFu);
   }
 }
 
@@ -80,7 +115,7 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant
 // ---------------------------------------------------------------------------
 template <bool BF16>
 __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_constant__ BwdArgs a) {
-  const int chunks = a.D / 8;
+  const int chunks = (a.D + 7) / 8;
   const int64_t n = (int64_t)a.H * a.rows * chunks;
   for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n;
        x += (int64_t)gridDim.x * blockDim.x) {
@@ -92,13 +127,40 @@ __global__ void __launch_bounds__(256) attn_dq_convert_kernel(const __grid_const
       const int32_t len = min(max(a.cu_q[row / a.Sq], 0), a.Sq);
       if (row % a.Sq >= len) continue;
     }
-    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + g * a.D + 8 * c);
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + g * a.DA + 8 * c);
     const float4 u = src[0], v = src[1];
     const float s = a.sm_scale;
     uint8_t* dst = reinterpret_cast<uint8_t*>(a.dq) +
                    2 * (row_offset(a.dq_stride, row, h, a.Sq, a.q_packed) + 8 * c);
-    st_global_v4(dst, pack2<BF16>(u.x * s, u.y * s), pack2<BF16>(u.z * s, u.w * s),
-                 pack2<BF16>(v.x * s, v.y * s), pack2<BF16>(v.z * s, v.w * s));
+    store_chunk8<BF16>(dst, u, v, s, a.D - 8 * c);
+  }
+}
+
+// The same for a stacked Q side whose sequences may leave rows unused
+// (lengths from seqused, positions from an array): block row b of the grid
+// converts sequence b's used rows only, so rows outside every sequence are
+// not written.
+template <bool BF16>
+__global__ void __launch_bounds__(256) attn_dq_convert_seq_kernel(const __grid_constant__ BwdArgs a) {
+  const int b = blockIdx.x;
+  int32_t row0, len;
+  stacked_bounds(a.cu_q, a.q_used ? a.used_q : nullptr, a.q_offsets != 0, b, a.total_q, &row0,
+                 &len);
+  const int chunks = (a.D + 7) / 8;
+  const int64_t n = (int64_t)a.H * len * chunks;
+  for (int64_t x = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; x < n;
+       x += (int64_t)gridDim.y * blockDim.x) {
+    const int c = (int)(x % chunks);
+    const int64_t hr = x / chunks;
+    const int h = (int)(hr / len);
+    const int64_t row = row0 + hr % len;
+    const int64_t g = (int64_t)h * a.rows + row;
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + g * a.DA + 8 * c);
+    const float4 u = src[0], v = src[1];
+    const float s = a.sm_scale;
+    uint8_t* dst = reinterpret_cast<uint8_t*>(a.dq) +
+                   2 * (row_offset(a.dq_stride, row, h, a.Sq, true) + 8 * c);
+    store_chunk8<BF16>(dst, u, v, s, a.D - 8 * c);
   }
 }
 
@@ -145,9 +207,13 @@ struct BwdCfg {
   static constexpr int kOffX = kOffDQ + kDqStageBytes;
   static constexpr int kOffBar = kOffX + 3 * kXBytes;
   // kv_full, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
-  // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done, x_ready
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 8;
-  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done, x_ready,
+  // delta_ready[2]
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 10;
+  // With dropout, delta is not folded into dP^T: each P/dS group stages the
+  // delta values of its 64 query columns, two tiles deep.
+  static constexpr int kOffDelta = kOffBar + 8 * kNumBars;
+  static constexpr int kOffMisc = kOffDelta + 2 * 2 * 64 * 4;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + DPAD;
   static constexpr bool kAliasDQ = (DPAD == 128);  // dQ tile reuses the dP^T columns
@@ -195,7 +261,7 @@ __device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t
   }
 }
 
-template <int DPAD, bool BF16>
+template <int DPAD, bool BF16, bool DROPOUT>
 __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<DPAD>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -209,15 +275,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   // Q and K sides are addressed independently (see the forward kernel).
   int32_t sq = a.Sq, sk = a.Sk, qrow0 = 0, krow0 = 0, bq = b, bk = b;
   if (a.q_packed) {
-    qrow0 = a.cu_q[b];
-    sq = a.cu_q[b + 1] - qrow0;
+    stacked_bounds(a.cu_q, a.q_used ? a.used_q : nullptr, a.q_offsets != 0, b, a.total_q, &qrow0, &sq);
     bq = 0;
   } else if (a.q_padded) {
     sq = min(max(a.cu_q[b], 0), a.Sq);
   }
   if (a.k_packed) {
-    krow0 = a.cu_k[b];
-    sk = a.cu_k[b + 1] - krow0;
+    stacked_bounds(a.cu_k, a.k_used ? a.used_k : nullptr, a.k_offsets != 0, b, a.total_k, &krow0, &sk);
     bk = 0;
   } else if (a.k_padded) {
     sk = min(max(a.cu_k[b], 0), a.Sk);
@@ -243,10 +307,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   if (n_it <= 0) {
     // No query sees these keys: dK = dV = 0.
     const int rows = min(128, sk - n0);
-    for (int idx = threadIdx.x; idx < rows * (a.D / 8); idx += blockDim.x) {
-      const int r = idx / (a.D / 8), c = idx % (a.D / 8);
-      st_global_v4(kv_row_ptr(a.dk, a.dk_stride, n0 + r) + 16 * c, 0u, 0u, 0u, 0u);
-      st_global_v4(kv_row_ptr(a.dv, a.dv_stride, n0 + r) + 16 * c, 0u, 0u, 0u, 0u);
+    for (int r = threadIdx.x / 4; r < rows; r += blockDim.x / 4) {
+      zero_row16(kv_row_ptr(a.dk, a.dk_stride, n0 + r), a.D, threadIdx.x & 3, 4);
+      zero_row16(kv_row_ptr(a.dv, a.dv_stride, n0 + r), a.Dv, threadIdx.x & 3, 4);
     }
     return;
   }
@@ -264,6 +327,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24,
                  dq_mma = s_full + 32, dq_free = s_full + 40, acc_done = s_full + 48,
                  x_ready = s_full + 56;
+  auto delta_ready = [&](int g) { return s_full + 64 + 8 * g; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -285,6 +349,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(dq_free, 128);
     mbar_init(acc_done, 1);
     mbar_init(x_ready, 256);
+    mbar_init(delta_ready(0), 128);
+    mbar_init(delta_ready(1), 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -349,12 +415,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     // P / dS warps work on tile it+1's P while dK(it) and dQ(it) run.
     if (lane == 0) {
       const uint32_t idesc_kk = make_idesc(BF16, 128, 128, false, false);   // S^T, dP^T
-      const uint32_t idesc_acc = make_idesc(BF16, 128, a.D, false, true);  // dV, dK (A in TMEM)
+      const uint32_t idesc_dv = make_idesc(BF16, 128, a.Dv16, false, true);  // dV (A in TMEM)
+      const uint32_t idesc_dk = make_idesc(BF16, 128, a.D16, false, true);   // dK (A in TMEM)
       // dQ: with a 128-wide head dim the transposed product dQ^T = K^T dS^T
       // (TMEM lane = head-dim index, column = query) lets the drain add whole
       // 128-byte rows; otherwise dQ = dS K (lane = query).
       const uint32_t idesc_dq = C::kDqTransposed ? make_idesc(BF16, 128, 128, true, true)
-                                                 : make_idesc(BF16, 128, a.D, true, true);
+                                                 : make_idesc(BF16, 128, a.D16, true, true);
       // Descriptor words: the high word is fixed per layout; the low word
       // carries the start address and is advanced by (bytes >> 4).
       const uint32_t hiK = (uint32_t)(make_sdesc(0, 16, 1024) >> 32);    // K-major
@@ -415,7 +482,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           // dV += P^T dO  (P^T from TMEM, dO MN-major)
           if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
           tc_fence_after();
-          bwd_issue_ts_halves(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_acc,
+          bwd_issue_ts_halves(tmem + C::kColDV, tmem + C::kColS, loDOm + dos * kTile16, hiM, idesc_dv,
                               it > 0);
           tc_commit(do_empty(dos));
           if (nx < n_it) {
@@ -429,7 +496,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           // dK += dS^T Q
           if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.status, kSiteMma))) break;
           tc_fence_after();
-          bwd_issue_ts_halves(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_acc,
+          bwd_issue_ts_halves(tmem + C::kColDK, tmem + C::kColDP, loQm + qs * kTile16, hiM, idesc_dk,
                               it > 0);
           tc_commit(q_empty(qs));
           // dQ tile (into the dP columns when aliased: in order after dK read them)
@@ -503,7 +570,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     const uint32_t xrow = (uint32_t)((r >> 3) * 256 + (r & 7) * 16);  // core matrix (r/8, 0)
     const float inv_c = 1.f / sl2;
     auto folded = [&](float v) -> float {
-      if (half == 1) return -v;
+      if (half == 1) return DROPOUT ? 0.f : -v;  // with dropout delta is applied per element
       return (v == -INFINITY || v == INFINITY || v != v) ? 0.f : -(v * 1.4426950408889634f) * inv_c;
     };
     auto put_row = [&](uint32_t base, float x) {
@@ -516,6 +583,51 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(base + xrow),
                    "r"((w_hi & 0xFFFFu) | (w_mid << 16)), "r"(w_lo & 0xFFFFu)
                    : "memory");
+    };
+    // Dropout: this group's delta values for tile `it` into its staging slot
+    // (threads 0-63 of the group write query columns qo .. qo + 63), then the
+    // group's delta_ready barrier.  Every thread of the group arrives once per
+    // tile and waits for that tile before reading, so the barrier never runs
+    // two phases ahead of a reader, and a slot is rewritten only two tiles
+    // later, after all of its readers have moved on.
+    const uint32_t sDelta = sbase + C::kOffDelta + half * 2 * 64 * 4;
+    auto stage_delta = [&](int it) {
+      if constexpr (DROPOUT) {
+        if (r < 64) {
+          const int32_t i = (mb + it) * 128 + qo + r;
+          float d = 0.f;
+          if (i < sq) {
+            const int64_t row = a.q_packed ? (int64_t)(qrow0 + i) : (int64_t)b * a.Sq + i;
+            d = a.delta[(int64_t)h * a.rows + row];
+          }
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(sDelta + (it & 1) * 256 + r * 4), "f"(d)
+                       : "memory");
+        }
+        mbar_arrive(delta_ready(half));
+      } else {
+        (void)it;
+      }
+    };
+    // Dropout: keep bits of this key row against the 32 query columns of
+    // chunk c of tile it.  Key j, query i take word (j mod 4) of Philox on the
+    // counter (j div 4, i, b H + h, offset).
+    const uint32_t bh = (uint32_t)(b * a.H + h);
+    auto keep_bits = [&](int it, int c) -> uint32_t {
+      uint32_t bits = 0;
+      if constexpr (DROPOUT) {
+        const uint32_t i0 = (uint32_t)((mb + it) * 128 + qo + 32 * c);
+        const int word = j & 3;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+          const uint4 wd = philox4x32_10(make_uint4((uint32_t)(j >> 2), i0 + k, bh, a.philox_offset),
+                                         a.seed_lo, a.seed_hi);
+          const uint32_t x = word == 0 ? wd.x : word == 1 ? wd.y : word == 2 ? wd.z : wd.w;
+          bits |= (x < a.keep_below ? 1u : 0u) << k;
+        }
+      } else {
+        (void)it, (void)c;
+      }
+      return bits;
     };
     {
       // Constant parts, then tile 0's terms; the MMA issuer waits on x_ready.
@@ -541,10 +653,15 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
-      // P is kept as the rounded 16-bit pairs the dV product uses.
+      // P is kept as the rounded 16-bit pairs the dV product uses (with
+      // dropout: the undropped P for dS, while the dV product gets the kept
+      // elements only; its factor 1 / (1 - p) is applied at the store).
       uint32_t pk[32];
+      uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+      if constexpr (DROPOUT) stage_delta(it);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
+        if constexpr (DROPOUT) keep[c] = keep_bits(it, c);
         uint32_t sr[32];
         tmem_ld32(tS + qo + 32 * c, sr);
         uint32_t chunk[16];
@@ -557,8 +674,14 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
             v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
             v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
           }
-          chunk[e] = pack2<BF16>(v0, v1);
-          pk[16 * c + e] = chunk[e];
+          pk[16 * c + e] = pack2<BF16>(v0, v1);
+          if constexpr (DROPOUT) {
+            v0 = (keep[c] >> (2 * e)) & 1u ? v0 : 0.f;
+            v1 = (keep[c] >> (2 * e + 1)) & 1u ? v1 : 0.f;
+            chunk[e] = pack2<BF16>(v0, v1);
+          } else {
+            chunk[e] = pk[16 * c + e];
+          }
         }
         tmem_st16(tS + po + 16 * c, chunk);
       }
@@ -573,20 +696,35 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       mbar_arrive(p_ready);
       // ---- phase 2: dS^T = P^T o (dP^T - delta), into TMEM and shared memory ----
       ok = mbar_wait(dp_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
-           (it == 0 || mbar_wait(dq_mma, (it - 1) & 1, abort_flag, a.status, kSiteSoftmax));
+           (it == 0 || mbar_wait(dq_mma, (it - 1) & 1, abort_flag, a.status, kSiteSoftmax)) &&
+           (!DROPOUT || mbar_wait(delta_ready(half), it & 1, abort_flag, a.status, kSiteSoftmax));
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
-        tmem_ld32(tDP + qo + 32 * c, dr);  // 32 queries of dP^T - delta
+        tmem_ld32(tDP + qo + 32 * c, dr);  // 32 queries of dP^T - delta (raw dP^T with dropout)
         uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 pe = unpack2<BF16>(pk[16 * c + e]);
-          const float d0 = pe.x * __uint_as_float(dr[2 * e]);
-          const float d1 = pe.y * __uint_as_float(dr[2 * e + 1]);
+          float d0, d1;
+          if constexpr (DROPOUT) {
+            // dS = P o (m s dP - delta): a dropped element keeps -P delta
+            float2 dl;
+            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                         : "=f"(dl.x), "=f"(dl.y)
+                         : "r"(sDelta + (it & 1) * 256 + (32 * c + 2 * e) * 4));
+            const float s0 = (keep[c] >> (2 * e)) & 1u ? a.drop_scale * __uint_as_float(dr[2 * e]) : 0.f;
+            const float s1 =
+                (keep[c] >> (2 * e + 1)) & 1u ? a.drop_scale * __uint_as_float(dr[2 * e + 1]) : 0.f;
+            d0 = pe.x * (s0 - dl.x);
+            d1 = pe.y * (s1 - dl.y);
+          } else {
+            d0 = pe.x * __uint_as_float(dr[2 * e]);
+            d1 = pe.y * __uint_as_float(dr[2 * e + 1]);
+          }
           dd[e] = pack2<BF16>(d0, d1);
         }
         tmem_st16(tDP + po + 16 * c, dd);
@@ -619,18 +757,16 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       uint8_t* row = valid ? (half == 0 ? kv_row_ptr(a.dv, a.dv_stride, j)
                                         : kv_row_ptr(a.dk, a.dk_stride, j))
                            : nullptr;
-      const float mul = half == 0 ? 1.f : a.sm_scale;
+      const float mul = half == 0 ? (DROPOUT ? a.drop_scale : 1.f) : a.sm_scale;
       const uint32_t tacc = tmem + lane_off + (half == 0 ? C::kColDV : C::kColDK);
-      for (int c = 0; c < a.D / 16; ++c) {
+      const int ncols = half == 0 ? a.Dv : a.D;  // dV has V's head dim, dK Q's
+      for (int c = 0; c < (ncols + 15) / 16; ++c) {
         uint32_t rv[16], pv[8];
         tmem_ld16(tacc + 16 * c, rv);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           pv[e] = pack2<BF16>(__uint_as_float(rv[2 * e]) * mul, __uint_as_float(rv[2 * e + 1]) * mul);
-        if (valid) {
-          st_global_v4(row + 32 * c, pv[0], pv[1], pv[2], pv[3]);
-          st_global_v4(row + 32 * c + 16, pv[4], pv[5], pv[6], pv[7]);
-        }
+        if (valid) st_row16(row, c, pv, ncols);
       }
     }
   } else {
@@ -652,6 +788,25 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       // outside the sequence hold exact zeros (their dS is 0), so whole boxes
       // can be added; columns past D are clipped by the tensor map.
       const int grow = (int)((int64_t)h * a.rows + row0);
+      // Deterministic mode: the key tiles that visit this query tile form one
+      // run [n_lo, ...]; this warp adds its column quarter of the tile after
+      // the n - n_lo key tiles before it have added theirs (a counter per
+      // head, tile and quarter), so every element's fp32 sum is taken in key
+      // tile order whatever order the CTAs run in.
+      int* order = a.order ? a.order + 4 * (int64_t)grow + quad : nullptr;
+      auto wait_turn = [&]() -> bool {  // called after the tile left TMEM
+        if (!order) return true;
+        int lo_n = 0, hi_n = ntile;  // smallest n' with m < m_end(n'), n' in [0, ntile]
+        while (lo_n < hi_n) {
+          const int mid = (lo_n + hi_n) >> 1;
+          int32_t mb2, me2;
+          bwd_tile_range(win, sq, sk, mid * 128, &mb2, &me2);
+          if (me2 > mb + it) hi_n = mid; else lo_n = mid + 1;
+        }
+        bool in_time = true;
+        if (lane == 0) in_time = wait_counter(order, ntile - lo_n, abort_flag, a.status, kSiteDq);
+        return __shfl_sync(0xffffffffu, in_time ? 1 : 0, 0) != 0;
+      };
       auto issue_box = [&](uint32_t buf, int col, int row) {
         fence_proxy_async_smem();
         __syncwarp();
@@ -678,6 +833,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         tmem_ld64(tDQ + 64, v1);
         tc_fence_before();
         mbar_arrive(dq_free);
+        if (!wait_turn()) break;
         if (active) {
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
@@ -693,24 +849,35 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         }
       } else {
         // lane = query row (this warp: rows 32 quad .. +31), TMEM column =
-        // head-dim index.  Each lane writes its row's 32 floats of a box.
-        for (int cc = 0; cc < (a.D + 31) / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tDQ + 32 * cc, v);
-          if (32 * cc + 32 >= a.D) {  // last chunk read: TMEM can be reused
-            tc_fence_before();
-            mbar_arrive(dq_free);
-          }
+        // head-dim index.  Each lane writes its row's 32 floats of a box.  The
+        // whole tile (at most 64 columns here) is read before any staging.
+        constexpr int kChunks = DPAD / 32;
+        uint32_t v[kChunks][32];
+#pragma unroll
+        for (int cc = 0; cc < kChunks; ++cc)
+          if (32 * cc < a.D) tmem_ld32(tDQ + 32 * cc, v[cc]);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        if (!wait_turn()) break;
+#pragma unroll
+        for (int cc = 0; cc < kChunks; ++cc) {
+          if (32 * cc >= a.D) break;
           const uint32_t buf = next_buf();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint32_t off = lane * 128 + (((uint32_t)k ^ (lane & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off), "r"(v[4 * k]),
-                         "r"(v[4 * k + 1]), "r"(v[4 * k + 2]), "r"(v[4 * k + 3])
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off),
+                         "r"(v[cc][4 * k]), "r"(v[cc][4 * k + 1]), "r"(v[cc][4 * k + 2]),
+                         "r"(v[cc][4 * k + 3])
                          : "memory");
           }
           issue_box(buf, 32 * cc, grow + 32 * quad);
         }
+      }
+      if (order && lane == 0) {
+        // this warp's additions are complete before the next key tile's
+        bulk_wait<0>();
+        release_counter(order);
       }
     }
     // The staged tiles must stay in place until the TMA has added them.
@@ -726,26 +893,19 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   }
 }
 
-template <int DPAD, bool BF16>
+template <int DPAD, bool BF16, bool DROPOUT>
 static cudaError_t launch_main(const BwdArgs& a, cudaStream_t stream) {
   using C = BwdCfg<DPAD>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   // One warp of each warpgroup per sub-partition: P/dS, P/dS, drain, TMA/MMA.
   static_assert(2 * C::kPdsRegs + C::kDrainRegs + C::kProducerRegs <= 4 * C::kLaunchRegs,
                 "register split exceeds the launch budget");
-  auto kern = attn_bwd_kernel<DPAD, BF16>;
-  // The setmaxnreg.inc of the P/dS and drain warpgroups draws on what the
-  // TMA/MMA warpgroup gives back from kLaunchRegs; with fewer registers at
-  // launch it would wait forever, so refuse to launch instead.
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs < C::kLaunchRegs) return cudaErrorLaunchOutOfResources;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  dim3 grid((a.Sk + 127) / 128, a.H, a.B);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(a);
-  return cudaGetLastError();
+  auto kern = attn_bwd_kernel<DPAD, BF16, DROPOUT>;
+  static std::atomic<uint64_t> prepared{0};
+  const dim3 grid((a.Sk + 127) / 128, a.H, a.B);
+  return prepared_launch(kern, prepared, a.dev, C::kSmemBytes, C::kLaunchRegs, [&] {
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(a);
+  });
 }
 
 template <bool BF16>
@@ -761,12 +921,24 @@ static cudaError_t launch_all(const BwdArgs& a, cudaStream_t stream, int sms) {
   if (a.Sk > 0 && a.H > 0 && a.B > 0) {
     cudaError_t e = cudaSuccess;
     if (a.main_events[0] && (e = cudaEventRecord(a.main_events[0], stream)) != cudaSuccess) return e;
-    e = a.D <= 64 ? launch_main<64, BF16>(a, stream) : launch_main<128, BF16>(a, stream);
+    // all tiles take the wider of the two head dims (TMA zero-fills the rest)
+    const bool narrow = a.D <= 64 && a.Dv <= 64;
+    if (a.dropout)
+      e = narrow ? launch_main<64, BF16, true>(a, stream) : launch_main<128, BF16, true>(a, stream);
+    else
+      e = narrow ? launch_main<64, BF16, false>(a, stream) : launch_main<128, BF16, false>(a, stream);
     if (e != cudaSuccess) return e;
     if (a.main_events[1] && (e = cudaEventRecord(a.main_events[1], stream)) != cudaSuccess) return e;
   }
+  if (groups > 0 && a.q_used) {
+    // per sequence: Sq (the largest seqlen_q) bounds each sequence's rows
+    const int64_t want = ((int64_t)a.H * a.Sq * ((a.D + 7) / 8) + 255) / 256;
+    const dim3 grid((unsigned)a.B, (unsigned)(want < 64 ? (want > 0 ? want : 1) : 64));
+    attn_dq_convert_seq_kernel<BF16><<<grid, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
   if (groups > 0) {
-    const int64_t n = groups * (a.D / 8);
+    const int64_t n = groups * ((a.D + 7) / 8);
     const int64_t want = (n + 255) / 256;
     const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
     attn_dq_convert_kernel<BF16><<<grid, 256, 0, stream>>>(a);
@@ -776,9 +948,7 @@ static cudaError_t launch_all(const BwdArgs& a, cudaStream_t stream, int sms) {
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = a.sms > 0 ? a.sms : 148;
   return a.bf16 ? launch_all<true>(a, stream, sms) : launch_all<false>(a, stream, sms);
 }
 

@@ -84,6 +84,37 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Ordered hand-over between CTAs through a global counter: wait (bounded,
+// like mbar_wait) until *ctr >= target, then order this thread's following
+// async-proxy operations (TMA reductions) after the observed writes.
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort,
+                                             uint32_t* status, uint32_t site) {
+  auto load = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    return v;
+  };
+  if (load() < target) {
+    const unsigned long long t0 = globaltimer();
+    while (load() < target) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(status, 1u << site);
+        return false;
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+// After this thread's TMA reductions have completed (cp.async.bulk.wait_group
+// 0): make them visible, then bump the counter with release semantics.
+__device__ __forceinline__ void release_counter(int* ctr) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // TMA: 4-D tiled load into shared memory, completion counted on an mbarrier.
 // Coordinates: x (innermost, elements), then rows, heads, batch.
@@ -329,6 +360,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC '11): ten rounds on a 128-bit counter, each two
+// 32 x 32 -> 64-bit products (multipliers 0xD2511F53 and 0xCD9E8D57) mixed
+// with the other counter words and the key, the key advanced by the Weyl
+// constants 0x9E3779B9 and 0xBB67AE85 between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c.x;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c.z;
+    const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
 // Two fp32 -> one packed pair of 16-bit floats, round to nearest even.
 // `lo` lands in the low half (the lower column / K index).
 template <bool BF16>
@@ -357,6 +409,39 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Stores 16 columns [16 c, 16 c + 16) of a row of 16-bit values (8 packed
+// pairs), only those below `ncols`; `row` is 16-byte aligned.
+__device__ __forceinline__ void st_row16(uint8_t* row, int c, const uint32_t (&pk)[8], int ncols) {
+  uint8_t* p = row + 32 * c;
+  if (16 * c + 16 <= ncols) {
+    st_global_v4(p, pk[0], pk[1], pk[2], pk[3]);
+    st_global_v4(p + 16, pk[4], pk[5], pk[6], pk[7]);
+    return;
+  }
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int col = 16 * c + 2 * w;
+    if (col + 1 < ncols)
+      *reinterpret_cast<uint32_t*>(p + 4 * w) = pk[w];
+    else if (col < ncols)
+      *reinterpret_cast<uint16_t*>(p + 4 * w) = (uint16_t)(pk[w] & 0xFFFFu);
+  }
+}
+// Zeroes the first `ncols` 16-bit values of a 16-byte aligned row; threads
+// `t` of `nt` share the work.
+__device__ __forceinline__ void zero_row16(uint8_t* row, int ncols, int t, int nt) {
+  for (int c = t; c < ncols / 8; c += nt) st_global_v4(row + 16 * c, 0u, 0u, 0u, 0u);
+  for (int col = (ncols / 8) * 8 + t; col < ncols; col += nt)
+    *reinterpret_cast<uint16_t*>(row + 2 * col) = 0;
+}
+
 // A compile-time flag passed to generic lambdas (for `if constexpr` code
 // paths instantiated per call site).
 template <bool V>
@@ -374,11 +459,22 @@ __device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0, int blocks
 #pragma unroll
       for (int c = 0; c < 8; ++c) st_shared_v4(tile + blk * 16384 + r * 128 + c * 16, 0u, 0u, 0u, 0u);
 }
-__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
+// Rows [*row0, *row0 + *len) of sequence b of a stacked (1THD) tensor with
+// `total` rows.  Positions: cu[b] (cumulative array, B + 1 entries, or an
+// array of B start rows when `offsets`); lengths: the cumulative difference,
+// or used[b] when `used` is given (capped by the slot cu[b + 1] - cu[b] of a
+// cumulative array).  Everything is clamped to [0, total]: an array that runs
+// past the tensor (an error of the caller) shortens the sequence instead of
+// sending reads and writes outside the tensor.
+__device__ __forceinline__ void stacked_bounds(const int32_t* cu, const int32_t* used,
+                                               bool offsets, int b, int64_t total,
+                                               int32_t* row0, int32_t* len) {
+  const int32_t t = (int32_t)total;  // total < 2^30 (checked on the host)
+  const int32_t a = min(max(cu[b], 0), t);
+  const int32_t z = offsets ? t : min(max(cu[b + 1], a), t);
+  *row0 = a;
+  *len = used ? min(max(used[b], 0), z - a) : z - a;
 }
+
 
 }  // namespace attn

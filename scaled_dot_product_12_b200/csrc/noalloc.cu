@@ -9,7 +9,6 @@
 #include <cuda_runtime.h>
 
 #include <cstring>
-#include <mutex>
 
 #include "../../include/attn.h"
 
@@ -17,30 +16,26 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_workspace[ATTN_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_ws_addr[kMaxDevices];  // device address of the array, per device (set once)
-
-// Device address of this device's copy of the array.  Host code cannot use
-// the symbol's name as a device pointer, so it is looked up once per device,
-// with that device current.
+// Device address of the stream's device's copy of the array.  Host code cannot
+// use the symbol's name as a device pointer, so the address is looked up with
+// that device current.  It is looked up on every call rather than cached: a
+// reset of the device's primary context reloads the module and can move the
+// array.
 cudaError_t workspace_address(cudaStream_t stream, void** out) {
   int cur = 0, dev = 0;
   cudaError_t e = cudaGetDevice(&cur);
   if (e != cudaSuccess) return e;
   dev = cur;
   if (stream != nullptr && (e = cudaStreamGetDevice(stream, &dev)) != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_ws_addr[dev] == nullptr) {
-    if (dev != cur && (e = cudaSetDevice(dev)) != cudaSuccess) return e;
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_workspace);
-    if (dev != cur) cudaSetDevice(cur);
-    if (e != cudaSuccess) return e;
-    g_ws_addr[dev] = p;
+  if (dev != cur && (e = cudaSetDevice(dev)) != cudaSuccess) return e;
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_static_workspace);
+  if (dev != cur) {
+    const cudaError_t r = cudaSetDevice(cur);  // the caller's device comes back either way
+    if (e == cudaSuccess) e = r;
   }
-  *out = g_ws_addr[dev];
+  if (e != cudaSuccess) return e;
+  *out = p;
   return cudaSuccess;
 }
 

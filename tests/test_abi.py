@@ -70,7 +70,7 @@ def _fwd(lib_b, **kw):
     B = lib_b
     p = B.FwdParams()
     p.struct_size = ctypes.sizeof(p)
-    p.version = 1
+    p.version = 2
     p.dtype = B.DTYPE_BF16
     p.B, p.H, p.Sq, p.Sk, p.D = 2, 3, 100, 90, 64
     p.q = p.k = p.v = p.o = p.lse = FAKE
@@ -89,18 +89,57 @@ def _call_fwd(B, p):
 
 
 @pytest.mark.parametrize("field,value", [
-    ("struct_size", 8), ("version", 2), ("dtype", 2), ("D", 72), ("D", 144), ("D", 0),
+    ("struct_size", 8), ("version", 3), ("version", 1), ("dtype", 2), ("D", 144), ("D", 0),
+    ("D", -3),
     ("B", -1), ("Sq", 1 << 30), ("sm_scale", float("nan")), ("sm_scale", float("inf")),
     ("varlen_bits", 1 << 19), ("varlen_bits", 1 << 31), ("varlen_bits", 0x20),
     ("varlen_bits", 0x2000), ("varlen_bits", 2 << 16), ("varlen_bits", 3 << 16),
     ("varlen_bits", 0x0B),                       # packed Q without cu_seqlens_q
-    ("varlen_bits", 0x0505),                     # length = array: not supported
+    ("varlen_bits", 0x0505),                     # stacked, length array, uniform positions
+    ("varlen_bits", 0x1313),                     # stacked, cumulative lengths, position array
+    ("flags", 1), ("flags", 2), ("Dv", -1), ("Dv", 129), ("dropout_p", -0.1), ("dropout_p", 1.0),
+    ("dropout_p", float("nan")),
     ("q", 0), ("o", 0), ("k", 0), ("q", FAKE + 8), ("o", FAKE + 2),
     ("q_stride", (3 * 128 * 64, 128 * 64, 60)),  # row stride of 120 bytes
     ("k_stride", (3 * 128 * 64, 0, 64)),         # zero head stride with H > 1
 ])
 def test_forward_rejects_invalid_parameters(B, field, value):
     assert _call_fwd(B, _fwd(B, **{field: value})) == B.ERROR_INVALID_VALUE
+
+
+def test_version_one_callers_are_accepted(B):
+    # a caller built against version 1 passes version 1 and the version-1 size:
+    # the call validates (an empty problem succeeds without a device) ...
+    p = _fwd(B, B=0, version=1, struct_size=B.FWD_PARAMS_V1_SIZE)
+    assert _call_fwd(B, p) == 0
+    # ... and the version-2 fields it cannot know are not read
+    p = _fwd(B, B=0, version=1, struct_size=B.FWD_PARAMS_V1_SIZE, flags=7, Dv=-5)
+    assert _call_fwd(B, p) == 0
+    q = _bwd(B, B=0, version=1, struct_size=B.BWD_PARAMS_V1_SIZE)
+    assert B.lib().attn_bwd(ctypes.byref(q), None) == 0
+    assert B.lib().attn_bwd_workspace_size(ctypes.byref(_bwd(B, version=1,
+                                                            struct_size=B.BWD_PARAMS_V1_SIZE))) \
+        == B.lib().attn_bwd_workspace_size(ctypes.byref(_bwd(B)))
+
+
+def test_header_version_one_sizes_match_the_binding(B):
+    text = open(HEADER).read()
+    assert "offsetof(attn_fwd_params, seqused_q)" in text
+    assert "offsetof(attn_bwd_params, seqused_q)" in text
+    assert B.FwdParams.seqused_q.offset == B.FWD_PARAMS_V1_SIZE
+    assert B.BwdParams.seqused_q.offset == B.BWD_PARAMS_V1_SIZE
+
+
+@pytest.mark.parametrize("mode_name", ["MODE_PACKED_USED", "MODE_PACKED_OFFSETS"])
+def test_used_length_modes_need_their_arrays(B, mode_name):
+    mode = getattr(B, mode_name)
+    bits = B.varlen_bits(mode, B.MODE_DENSE, 0, 0)
+    p = _fwd(B, varlen_bits=bits, total_q=100, cu_seqlens_q=FAKE)   # no seqused_q
+    p.q_stride = p.o_stride = (0, 64, 3 * 64)
+    assert _call_fwd(B, p) == B.ERROR_INVALID_VALUE
+    p = _fwd(B, varlen_bits=bits, total_q=100, seqused_q=FAKE)      # no positions
+    p.q_stride = p.o_stride = (0, 64, 3 * 64)
+    assert _call_fwd(B, p) == B.ERROR_INVALID_VALUE
 
 
 def test_reserved_diagonal_bits_rejected_but_diagonal_accepted_in_validation(B):
@@ -126,7 +165,7 @@ def _bwd(lib_b, **kw):
     B = lib_b
     p = B.BwdParams()
     p.struct_size = ctypes.sizeof(p)
-    p.version = 1
+    p.version = 2
     p.dtype = B.DTYPE_FP16
     p.B, p.H, p.Sq, p.Sk, p.D = 2, 3, 100, 90, 128
     for n in ("q", "k", "v", "o", "dout", "lse", "dq", "dk", "dv", "workspace"):
@@ -222,3 +261,24 @@ def test_allowed_pairs_matches_oracle_count(B, w, sq, sk):
     if sq * sk > 2e7 and w[0] not in (INF, CTL):
         pytest.skip("large sizes only for the two common windows")
     assert B.allowed_pairs(sq, sk, *w) == ref.allowed_count(sq, sk, *w)
+
+
+@pytest.mark.parametrize("w", PLAN_WINDOWS + [(-500, 600, 0), (-130, 2, 1), (700, -650, 0)])
+@pytest.mark.parametrize("sq,sk", PLAN_SIZES + [(1000, 300), (300, 1000)])
+def test_key_tiles_visiting_a_query_tile_are_contiguous(B, w, sq, sk):
+    # The deterministic backward orders the dQ contributions of one query tile
+    # by key tile and gives each key tile the rank n - n_lo, n_lo found by
+    # bisection on "m < m_end(n)": that needs the visiting key tiles to form
+    # one run, and every key tile below a visiting one to have m_end <= m or
+    # to visit too.
+    plans = [B.tile_plan_bwd(sq, sk, w[0], w[1], w[2], n0) for n0 in range(0, sk, 128)]
+    for m in range(0, (sq + 127) // 128):
+        visit = [mb <= m < me for mb, me in plans]
+        ns = [n for n, v in enumerate(visit) if v]
+        if not ns:
+            continue
+        assert ns == list(range(ns[0], ns[-1] + 1)), (m, ns)
+        for n in range(ns[0]):
+            assert plans[n][1] <= m, (m, n, plans[n])
+        for n in ns:
+            assert plans[n][1] > m

@@ -38,7 +38,7 @@ def test_padded_mode_encoding_matches_header():
 def _fwd_params(B, bits, with_lengths):
     p = B.FwdParams()
     p.struct_size = ctypes.sizeof(p)
-    p.version = 1
+    p.version = B.PARAMS_VERSION
     p.dtype = B.DTYPE_BF16
     p.B, p.H, p.Sq, p.Sk, p.D = 2, 3, 100, 90, 64
     fake = 0x7F0000000000  # never dereferenced: validation fails first
@@ -89,7 +89,7 @@ def test_padded_workspace_matches_dense():
     for mode in (B.MODE_DENSE, B.MODE_PADDED):
         p = B.BwdParams()
         p.struct_size = ctypes.sizeof(p)
-        p.version = 1
+        p.version = B.PARAMS_VERSION
         p.dtype = B.DTYPE_BF16
         p.B, p.H, p.Sq, p.Sk, p.D = 3, 2, 300, 357, 128
         p.sm_scale = 0.1
