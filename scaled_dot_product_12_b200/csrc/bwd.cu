@@ -343,14 +343,14 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_ready, 256);
-    mbar_init(ds_ready, 256);
+    mbar_init(p_ready, 8);  // one arrival per P/dS warp
+    mbar_init(ds_ready, 8);
     mbar_init(dq_mma, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(dq_free, 4);  // one per drain warp
     mbar_init(acc_done, 1);
-    mbar_init(x_ready, 256);
-    mbar_init(delta_ready(0), 128);
-    mbar_init(delta_ready(1), 128);
+    mbar_init(x_ready, 8);
+    mbar_init(delta_ready(0), 4);  // one per warp of the group
+    mbar_init(delta_ready(1), 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -399,13 +399,11 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         ++ndo;
       }
       if (*abort_flag) {
-        mbar_wait(kv_full, 0, abort_flag, a.status, kSiteTeardown);
+        mbar_drain(kv_full, 0, a.status);
         for (int it = max(0, nq - C::kQStages); it < nq; ++it)
-          mbar_wait(q_full(it % C::kQStages), (it / C::kQStages) & 1, abort_flag, a.status,
-                    kSiteTeardown);
+          mbar_drain(q_full(it % C::kQStages), (it / C::kQStages) & 1, a.status);
         for (int it = max(0, ndo - C::kDOStages); it < ndo; ++it)
-          mbar_wait(do_full(it % C::kDOStages), (it / C::kDOStages) & 1, abort_flag, a.status,
-                    kSiteTeardown);
+          mbar_drain(do_full(it % C::kDOStages), (it / C::kDOStages) & 1, a.status);
       }
     }
   } else if (warp == C::kMmaWarp) {
@@ -439,12 +437,15 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       const uint64_t dXA = make_sdesc_plain(sXA, 128, 256), dXQ = make_sdesc_plain(sXQ, 128, 256),
                      dXD = make_sdesc_plain(sXD, 128, 256);
       // The issue loop is instantiated twice, with the padding clears (some
-      // side is padded) and without them, so dense and packed calls run code
-      // that carries no trace of the clears.
+      // side leaves rows unused: padded, or stacked with used lengths) and
+      // without them, so dense and packed calls run code that carries no
+      // trace of the clears.
       auto issue_all = [&](auto padding) {
-        // Padded batches: tile rows past seqlen_q / seqlen_k hold the caller's
-        // padding, not TMA zero fill; P and dS are 0 there, but 0 * NaN is not,
-        // so those rows are zeroed before the tensor cores first read a tile.
+        // Tile rows past seqlen_q / seqlen_k may hold the caller's padding (a
+        // padded batch, the unused rows of a slot, a gap between stacked
+        // sequences), not TMA zero fill; P and dS are 0 there, but 0 * NaN is
+        // not, so those rows are zeroed before the tensor cores first read a
+        // tile.
         auto clear_padding = [&](bool side_padded, uint32_t tile, int r0) {
           if constexpr (decltype(padding)::value) {
             if (side_padded && r0 < 128) {
@@ -459,9 +460,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
                   mbar_wait(q_full(0), 0, abort_flag, a.status, kSiteMma) &&
                   mbar_wait(x_ready, 0, abort_flag, a.status, kSiteMma);
         if (ok) {
-          clear_padding(a.k_padded, sK, sk - n0);
-          clear_padding(a.k_padded, sV, sk - n0);
-          clear_padding(a.q_padded, sQ, sq - mb * 128);
+          clear_padding(a.k_padded || a.k_used, sK, sk - n0);
+          clear_padding(a.k_padded || a.k_used, sV, sk - n0);
+          clear_padding(a.q_padded || a.q_used, sQ, sq - mb * 128);
           tc_fence_after();
           bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ, hiK, idesc_kk);
           mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           ok = mbar_wait(do_full(0), 0, abort_flag, a.status, kSiteMma);
         }
         if (ok) {
-          clear_padding(a.q_padded, sDO, sq - mb * 128);
+          clear_padding(a.q_padded || a.q_used, sDO, sq - mb * 128);
           tc_fence_after();
           bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO, hiK, idesc_kk);
           mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           tc_commit(do_empty(dos));
           if (nx < n_it) {
             if (!(ok = mbar_wait(q_full(nqs), npar, abort_flag, a.status, kSiteMma))) break;
-            clear_padding(a.q_padded, sQ + nqs * C::kTileBytes, sq - (mb + nx) * 128);
+            clear_padding(a.q_padded || a.q_used, sQ + nqs * C::kTileBytes, sq - (mb + nx) * 128);
             tc_fence_after();
             bwd_issue_kmajor<DPAD / 16>(tmem + C::kColS, loK, loQ + nqs * kTile16, hiK, idesc_kk);
             mma_ss(tmem + C::kColS, dXA, dXQ, idesc_x, true);
@@ -512,7 +513,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
             if (!(ok = mbar_wait(do_full(ndos), ndpar, abort_flag, a.status, kSiteMma))) break;
             if (C::kAliasDQ && !(ok = mbar_wait(dq_free, it & 1, abort_flag, a.status, kSiteMma)))
               break;
-            clear_padding(a.q_padded, sDO + ndos * C::kTileBytes, sq - (mb + nx) * 128);
+            clear_padding(a.q_padded || a.q_used, sDO + ndos * C::kTileBytes, sq - (mb + nx) * 128);
             tc_fence_after();
             bwd_issue_kmajor<DPAD / 16>(tmem + C::kColDP, loV, loDO + ndos * kTile16, hiK, idesc_kk);
             mma_ss(tmem + C::kColDP, dXA, dXD, idesc_x, true);
@@ -520,8 +521,11 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           }
         }
         tc_commit(acc_done);
+        // every MMA issued has completed before TMEM can be released (on an
+        // abort too, when the other warps skip their wait on acc_done)
+        mbar_drain(acc_done, 0, a.status);
       };
-      if (a.q_padded || a.k_padded)
+      if (a.q_padded || a.k_padded || a.q_used || a.k_used)
         issue_all(Flag<true>{});
       else
         issue_all(Flag<false>{});
@@ -586,10 +590,10 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     };
     // Dropout: this group's delta values for tile `it` into its staging slot
     // (threads 0-63 of the group write query columns qo .. qo + 63), then the
-    // group's delta_ready barrier.  Every thread of the group arrives once per
-    // tile and waits for that tile before reading, so the barrier never runs
-    // two phases ahead of a reader, and a slot is rewritten only two tiles
-    // later, after all of its readers have moved on.
+    // group's delta_ready barrier.  Every warp of the group arrives once per
+    // tile (after all its lanes) and waits for that tile before reading, so
+    // the barrier never runs two phases ahead of a reader, and a slot is
+    // rewritten only two tiles later, after all of its readers have moved on.
     const uint32_t sDelta = sbase + C::kOffDelta + half * 2 * 64 * 4;
     auto stage_delta = [&](int it) {
       if constexpr (DROPOUT) {
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(sDelta + (it & 1) * 256 + r * 4), "f"(d)
                        : "memory");
         }
-        mbar_arrive(delta_ready(half));
+        mbar_arrive_warp(delta_ready(half));
       } else {
         (void)it;
       }
@@ -641,7 +645,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       st_shared_v4(xb + xrow + 128, 0u, 0u, 0u, 0u);
       put_row(xb, folded(row_val(0)));
       fence_proxy_async_smem();
-      mbar_arrive(x_ready);
+      mbar_arrive_warp(x_ready);
     }
     float v_next = n_it > 1 ? row_val(1) : 0.f;  // this group's value for tile it + 1
     bool ok = true;
@@ -693,7 +697,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive_warp(p_ready);
       // ---- phase 2: dS^T = P^T o (dP^T - delta), into TMEM and shared memory ----
       ok = mbar_wait(dp_full, it & 1, abort_flag, a.status, kSiteSoftmax) &&
            (it == 0 || mbar_wait(dq_mma, (it - 1) & 1, abort_flag, a.status, kSiteSoftmax)) &&
@@ -747,7 +751,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_ready);
+      mbar_arrive_warp(ds_ready);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, a.status, kSiteEpilogue));
     if (ok) {
@@ -832,7 +836,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         tmem_ld64(tDQ, v0);
         tmem_ld64(tDQ + 64, v1);
         tc_fence_before();
-        mbar_arrive(dq_free);
+        mbar_arrive_warp(dq_free);
         if (!wait_turn()) break;
         if (active) {
 #pragma unroll
@@ -857,7 +861,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         for (int cc = 0; cc < kChunks; ++cc)
           if (32 * cc < a.D) tmem_ld32(tDQ + 32 * cc, v[cc]);
         tc_fence_before();
-        mbar_arrive(dq_free);
+        mbar_arrive_warp(dq_free);
         if (!wait_turn()) break;
 #pragma unroll
         for (int cc = 0; cc < kChunks; ++cc) {

@@ -64,6 +64,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One arrival per warp on `bar`, whose count is the number of warps that
+// arrive: the warp barrier orders every lane's earlier work (its shared-memory
+// stores, and tcgen05 operations fenced with tc_fence_before) before lane 0's
+// arrival, and 32 lanes no longer contend for one mbarrier word.
+__device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Bounded wait on phase `parity`.  Returns false if the CTA was told to abort
 // (`*abort` set by another warp) or the time limit passed (then it records
 // `site` in *status and raises the CTA abort flag itself).
@@ -113,6 +122,20 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
 __device__ __forceinline__ void release_counter(int* ctr) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
+// Teardown wait on phase `parity`: bounded like mbar_wait but not cut short
+// by the CTA's abort flag, so that copies and MMAs already in flight land
+// before shared memory and TMEM are released.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return;
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(status, 1u << kSiteTeardown);
+      return;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

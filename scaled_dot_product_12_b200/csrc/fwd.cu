@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
     }
     for (int t = 0; t < NQ; ++t) {
       mbar_init(s_full(t), 1);
-      mbar_init(p_ready(t), 128);
+      mbar_init(p_ready(t), 4);  // one arrival per softmax warp
       mbar_init(o_done(t), 1);
     }
     for (int s = 0; s < C::kKStages; ++s) {
@@ -312,16 +312,13 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       if (*abort_flag) {
         // Drain: wait (bounded) for every copy still in flight.
         for (int64_t i = nk > C::kKStages ? nk - C::kKStages : 0; i < nk; ++i)
-          mbar_wait(k_full((int)(i % C::kKStages)), (uint32_t)((i / C::kKStages) & 1), abort_flag,
-                    args.status, kSiteTeardown);
+          mbar_drain(k_full((int)(i % C::kKStages)), (uint32_t)((i / C::kKStages) & 1), args.status);
         for (int64_t i = nv > C::kVStages ? nv - C::kVStages : 0; i < nv; ++i)
-          mbar_wait(v_full((int)(i % C::kVStages)), (uint32_t)((i / C::kVStages) & 1), abort_flag,
-                    args.status, kSiteTeardown);
+          mbar_drain(v_full((int)(i % C::kVStages)), (uint32_t)((i / C::kVStages) & 1), args.status);
         for (int qb = 0; qb < C::kQBufs; ++qb)
           for (int t = 0; t < NQ; ++t)
             if (qn[qb][t] > 0)
-              mbar_wait(q_full(qb, t), (uint32_t)((qn[qb][t] - 1) & 1), abort_flag, args.status,
-                        kSiteTeardown);
+              mbar_drain(q_full(qb, t), (uint32_t)((qn[qb][t] - 1) & 1), args.status);
       }
     }
   } else if (warp == C::kMmaWarp) {
@@ -338,9 +335,10 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       const uint32_t dQ = (uint32_t)make_sdesc(sQ, 16, 1024), dK = (uint32_t)make_sdesc(sK, 16, 1024);
       const uint32_t dV = (uint32_t)make_sdesc(sV, 16384, 1024);
       constexpr uint32_t kTile16 = C::kTileBytes >> 4;
-      // The unit loop is instantiated twice, with the V padding clears (K
-      // side padded) and without them, so other calls run code that carries
-      // no trace of the clears.
+      // The unit loop is instantiated twice, with the V padding clears (a K
+      // side whose sequences leave rows unused: padded, or stacked with used
+      // lengths) and without them, so other calls run code that carries no
+      // trace of the clears.
       auto run = [&](auto padding) {
         int64_t g = 0;        // key tiles of the units done so far
         int64_t gt[NQ] = {};  // the same, per query tile
@@ -352,9 +350,10 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
           if (!fwd_unit<NQ>(args, n_mblocks, units, u, w) || w.n_tiles <= 0) continue;
           const int qb = uc % C::kQBufs;
           ++uc;
-          // Padded batches: rows of a V tile past seqlen_k hold the caller's
-          // padding, not TMA zero fill; P is 0 there, but 0 * NaN is not, so
-          // the rows are zeroed before the tensor cores read the tile.
+          // Rows of a V tile past seqlen_k may hold the caller's padding (a
+          // padded batch, the unused rows of a slot or a gap between stacked
+          // sequences), not TMA zero fill; P is 0 there, but 0 * NaN is not,
+          // so the rows are zeroed before the tensor cores read the tile.
           auto clear_v_padding = [&](int it_v, int vs) {
             if constexpr (decltype(padding)::value) {
               const int r0 = w.sk - (w.nb + it_v) * 128;
@@ -434,13 +433,13 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
           for (int t = 0; t < w.nt; ++t) gt[t] += w.n_tiles;
         }
       };
-      if (args.k_padded)
+      if (args.k_padded || args.k_used)
         run(Flag<true>{});
       else
         run(Flag<false>{});
       // Everything issued has completed before TMEM is released.
       tc_commit(mma_done);
-      mbar_wait(mma_done, 0, abort_flag, args.status, kSiteTeardown);
+      mbar_drain(mma_done, 0, args.status);
     }
   }
   } else {
@@ -578,7 +577,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_ready(t));
+        mbar_arrive_warp(p_ready(t));
       }
       if (ok) {
         ok = mbar_wait(o_done(t), (uint32_t)((g + w.n_tiles - 1) & 1), abort_flag, args.status,
