@@ -465,8 +465,11 @@ def load_traffic(kernel, workload):
 def e2e_groups(w: synth.Workload, n_groups: int):
     """Slices along which the end-to-end step is pipelined: batches when there
     are several (LSE rows of a batch are contiguous in HT layout), else heads
-    of the single batch; packed workloads run as one group."""
-    if w.packed or n_groups <= 1:
+    of the single batch.  Packed workloads, and steps whose inputs are under
+    64 MB (latency-bound: more calls would only add host time), run as one
+    group."""
+    in_bytes = 2 * w.D * w.H * w.B * (2 * w.Sq + 2 * w.Sk)
+    if w.packed or n_groups <= 1 or in_bytes < (64 << 20):
         return None, [slice(None)]
     dim, size = (0, w.B) if w.B > 1 else (1, w.H)
     n = min(n_groups, size)

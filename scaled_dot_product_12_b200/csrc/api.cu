@@ -322,6 +322,8 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
     a.lse_th = m.lse_th;
     a.bf16 = p->dtype == ATTN_DTYPE_BF16;
     a.negate = p->sm_scale < 0.f;
+    // unit costs differ under any window; equal without one
+    a.units_by_cost = !(p->window_left == ATTN_WINDOW_INF && p->window_right == ATTN_WINDOW_INF);
     a.total_q = p->total_q;
     a.total_k = p->total_k;
     a.scale_log2 = std::fabs(p->sm_scale) * 1.4426950408889634f;

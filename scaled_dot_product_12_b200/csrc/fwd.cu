@@ -97,10 +97,15 @@ struct FwdUnit {
   SeqWindow win;
 };
 
-// The unit list: n_full units of NQ tiles, numbered query block fastest
-// (last block first), then head, then sequence, so the CTAs that run at the
-// same time work on the query blocks of a few heads and share those heads' K
-// and V tiles in L2.  Dealt round robin to G CTAs, they fill n_full / G whole
+// The unit list: n_full units of NQ tiles.  Without a mask every unit costs
+// the same, and units are numbered query block fastest (last block first),
+// then head, then sequence, so the CTAs that run at the same time work on the
+// query blocks of a few heads and share those heads' K and V tiles in L2.
+// Under a window the cost of a unit depends on its query block (a causal
+// mask gives the last block of a head the most key tiles), and units are
+// numbered query block slowest, last block first: dealt round robin, the
+// most expensive units go out first and every CTA gets a mix (longest
+// processing time first).  Dealt to G CTAs, the units fill n_full / G whole
 // rounds and a last, partial one; when the units of that last round number
 // at most G / 2, each is split into its NQ = 2 query tiles, units of one
 // tile, so the last round takes about half as long.
@@ -132,8 +137,16 @@ __device__ __forceinline__ bool fwd_unit(const FwdArgs& a, int32_t n_mblocks, co
     half = (int32_t)((u - us.split_from) & 1);
     w.nt = 1;
   }
-  const int64_t hb = fu / n_mblocks;
-  const int32_t mrev = (int32_t)(fu - hb * n_mblocks);
+  int64_t hb;
+  int32_t mrev;
+  if (a.units_by_cost) {
+    const int64_t HB = (int64_t)a.H * a.B;
+    mrev = (int32_t)(fu / HB);
+    hb = fu - (int64_t)mrev * HB;
+  } else {
+    hb = fu / n_mblocks;
+    mrev = (int32_t)(fu - hb * n_mblocks);
+  }
   w.h = (int32_t)(hb % a.H);
   w.b = (int32_t)(hb / a.H);
   // Q and K sides are addressed independently: packed (rows from the

@@ -23,6 +23,7 @@ struct FwdArgs {
   int32_t D16;  // D rounded up to 16 (MMA N; the columns past D are zero)
   int32_t Dv, Dv16;  // head dim of V and O, and rounded up to 16
   int32_t wl, wr, bottom_right, lse_th, bf16, negate;
+  int32_t units_by_cost;  // number units query block slowest (any mask), else fastest
   // Per side (Q: Q, O, LSE; K: K, V): stacked 1THD (positions in cu_q / cu_k:
   // B + 1 cumulative entries, or B start rows with *_offsets; lengths from
   // the cumulative differences, or from used_q / used_k with *_used), or

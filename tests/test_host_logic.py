@@ -152,7 +152,7 @@ def test_traffic_is_null_for_other_kernel_builds(tmp_path, monkeypatch):
 def test_end_to_end_groups_cover_the_workload_once():
     for name, w in synth.ALL_WORKLOADS.items():
         dim, groups = bench.e2e_groups(w, 4)
-        if w.packed:
+        if w.packed or name == "tiny_causal":
             assert dim is None and groups == [slice(None)]
             continue
         size = w.B if dim == 0 else w.H
