@@ -31,6 +31,12 @@ section "Bottom-Right Aligned Sliding Windows": a numeric window becomes
 L = wl - d, R = wr + d with d = seqlen_k - seqlen_q taken per sequence;
 sentinel windows are never shifted).
 
+Additive bias (the AOTriton 0.10b release notes, "Known Problems", and the
+0.14b notes, "Kernel Bug Fixes", where the bias is converted to fp32 before
+it is added): an optional matrix B [Sq, Sk] per (sequence, head) enters the
+logits, S_ij = c * <q_i, k_j> + B_ij on allowed (i, j) only (a bias never
+unmasks a pair); its gradient is dB = dS.
+
 Readings where the pages are silent:
   * a row i may attend key j iff j >= i - L and j <= i + R, both ends
     inclusive, an unbounded side imposing nothing;
@@ -124,9 +130,12 @@ def row_extent(seqlen_q, seqlen_k, window_left, window_right, bottom_right):
     return lo, hi, cnt
 
 
-def _probs_block(q, k, sm_scale, mask):
-    """P and LSE for a block of rows (fp64), fully masked rows -> 0 / -inf."""
+def _probs_block(q, k, sm_scale, mask, bias=None):
+    """P and LSE for a block of rows (fp64), fully masked rows -> 0 / -inf;
+    ``bias`` [rows, Sk] is added to the scaled scores."""
     s = sm_scale * (q @ k.T)
+    if bias is not None:
+        s = s + np.asarray(bias, dtype=np.float64)
     nonempty = mask.any(axis=1)
     m = np.where(mask, s, -np.inf).max(axis=1, initial=-np.inf)
     m = np.where(nonempty, m, 0.0)
@@ -137,11 +146,13 @@ def _probs_block(q, k, sm_scale, mask):
     return p, lse
 
 
-def forward(q, k, v, sm_scale, window_left, window_right, bottom_right=False, rows=None):
+def forward(q, k, v, sm_scale, window_left, window_right, bottom_right=False, rows=None,
+            bias=None):
     """One (sequence, head): q [Sq, D], k [Sk, D], v [Sk, Dv] -> (O, LSE).
 
     ``rows`` (optional) computes only those query rows (each row of the
     definition depends on its own query only) and returns [len(rows), ...].
+    ``bias`` (optional) [Sq, Sk] is added to the scaled scores.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -154,7 +165,8 @@ def forward(q, k, v, sm_scale, window_left, window_right, bottom_right=False, ro
         r1 = min(r0 + ROW_BLOCK, len(idx))
         sel = idx[r0:r1]
         mask = allowed(sq, sk, window_left, window_right, bottom_right, sel)
-        p, lse[r0:r1] = _probs_block(q[sel], k, sm_scale, mask)
+        p, lse[r0:r1] = _probs_block(q[sel], k, sm_scale, mask,
+                                     None if bias is None else np.asarray(bias)[sel])
         o[r0:r1] = p @ v
     return o, lse
 
@@ -175,8 +187,10 @@ def delta(o, do):
 
 
 def backward(q, k, v, do, sm_scale, window_left, window_right, bottom_right=False,
-             rows=None):
-    """One (sequence, head): gradient of <dO, O> -> (dQ, dK, dV).
+             rows=None, bias=None):
+    """One (sequence, head): gradient of <dO, O> -> (dQ, dK, dV), or
+    (dQ, dK, dV, dBias) when ``bias`` [Sq, Sk] is given (dBias = dS, zero on
+    masked pairs).
 
     ``rows`` (optional) restricts dQ to those query rows; dK and dV always sum
     over every query row (they need all of them).
@@ -189,10 +203,12 @@ def backward(q, k, v, do, sm_scale, window_left, window_right, bottom_right=Fals
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
+    db = None if bias is None else np.zeros((sq, sk), dtype=np.float64)
     for r0 in range(0, sq, ROW_BLOCK):
         r1 = min(r0 + ROW_BLOCK, sq)
         mask = allowed(sq, sk, window_left, window_right, bottom_right, np.arange(r0, r1))
-        p, _ = _probs_block(q[r0:r1], k, sm_scale, mask)
+        p, _ = _probs_block(q[r0:r1], k, sm_scale, mask,
+                            None if bias is None else np.asarray(bias)[r0:r1])
         o_blk = p @ v
         dv += p.T @ do[r0:r1]
         dp = do[r0:r1] @ v.T
@@ -200,8 +216,12 @@ def backward(q, k, v, do, sm_scale, window_left, window_right, bottom_right=Fals
         ds = p * (dp - dlt[:, None])
         dq[r0:r1] = sm_scale * (ds @ k)
         dk += sm_scale * (ds.T @ q[r0:r1])
+        if db is not None:
+            db[r0:r1] = ds
     if rows is not None:
         dq = dq[np.asarray(rows)]
+    if db is not None:
+        return dq, dk, dv, db
     return dq, dk, dv
 
 

@@ -461,3 +461,111 @@ def test_planted_dense_wrapper_index_slips_are_caught():
         _check_dense_wrappers(_planted_forward_dense_wrong_head, ref.backward_dense, w)
     with pytest.raises(AssertionError):
         _check_dense_wrappers(ref.forward_dense, _planted_backward_dense_batch_swap, w)
+
+
+# ---------------------------------------------------------------------------
+# Additive bias (AOTriton 0.10b "Known Problems", 0.14b "Kernel Bug Fixes"):
+# logits c <q_i, k_j> + B_ij on allowed pairs, dB = dS.
+# ---------------------------------------------------------------------------
+
+BIAS_WINDOWS = [(INF, INF, False), (CTL, 0, False), (2, 1, True), (CBR, 0, True), (3, -2, False)]
+
+
+def _brute_bias(q, k, v, do, c, w, bias):
+    """Independent formulation: dense mask, torch softmax over c QK^T + B,
+    autograd for every input including the bias."""
+    sq, sk = q.shape[0], k.shape[0]
+    wl, wr, br = w
+    d = sk - sq
+    mask = torch.zeros(sq, sk, dtype=torch.bool)
+    for i in range(sq):
+        for j in range(sk):
+            if wl == CTL:
+                ok = j <= i
+            elif wl == CBR:
+                ok = j <= i + d
+            else:
+                lo_ok = True if wl == INF else (j >= i - (wl - d if br else wl))
+                hi_ok = True if wr == INF else (j <= i + (wr + d if br else wr))
+                ok = lo_ok and hi_ok
+            mask[i, j] = ok
+    tq, tk, tv, tb = (torch.tensor(a, dtype=torch.float64, requires_grad=True)
+                      for a in (q, k, v, bias))
+    s = (tq @ tk.T) * c + tb
+    s = s.masked_fill(~mask, float("-inf"))
+    rows = mask.any(1)
+    lse = torch.logsumexp(s, dim=1)
+    o = torch.zeros(sq, v.shape[1], dtype=torch.float64)
+    if rows.any():
+        p = torch.softmax(s[rows], dim=1)
+        o = o.index_put((rows.nonzero()[:, 0],), p @ tv)
+    ((o * torch.tensor(do)).sum() + 0.0 * (tq.sum() + tk.sum() + tv.sum() + tb.sum())).backward()
+    return (o.detach().numpy(), lse.detach().numpy(), tq.grad.numpy(), tk.grad.numpy(),
+            tv.grad.numpy(), tb.grad.numpy())
+
+
+@pytest.mark.parametrize("w", BIAS_WINDOWS)
+@pytest.mark.parametrize("c", [0.6, -0.3])
+def test_bias_matches_independent_brute_force(w, c):
+    sq, sk, d = 6, 9, 4
+    q, k, v, do = (_rand(s, 60 + i) for i, s in enumerate([(sq, d), (sk, d), (sk, d), (sq, d)]))
+    bias = 2.0 * _rand((sq, sk), 70)
+    o, lse = ref.forward(q, k, v, c, *w, bias=bias)
+    dq, dk, dv, db = ref.backward(q, k, v, do, c, *w, bias=bias)
+    bo, blse, bdq, bdk, bdv, bdb = _brute_bias(q, k, v, do, c, w, bias)
+    np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(blse))
+    fin = np.isfinite(blse)
+    np.testing.assert_allclose(lse[fin], blse[fin], rtol=1e-12, atol=1e-12)
+    for a, b in ((dq, bdq), (dk, bdk), (dv, bdv), (db, bdb)):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("w", BIAS_WINDOWS[:3])
+def test_bias_gradient_matches_central_differences(w):
+    sq, sk, d = 5, 7, 3
+    q, k, v, do = (_rand(s, 80 + i) for i, s in enumerate([(sq, d), (sk, d), (sk, d), (sq, d)]))
+    bias = _rand((sq, sk), 90)
+    *_, db = ref.backward(q, k, v, do, 0.7, *w, bias=bias)
+
+    def loss(b):
+        o, _ = ref.forward(q, k, v, 0.7, *w, bias=b)
+        return float((o * do).sum())
+    h = 1e-6
+    num = np.zeros_like(bias)
+    for idx in np.ndindex(bias.shape):
+        old = bias[idx]
+        bias[idx] = old + h
+        fp = loss(bias)
+        bias[idx] = old - h
+        fm = loss(bias)
+        bias[idx] = old
+        num[idx] = (fp - fm) / (2 * h)
+    np.testing.assert_allclose(db, num, rtol=1e-6, atol=1e-7)
+    assert np.all(db[~ref.allowed(sq, sk, *w)] == 0)
+
+
+def test_bias_constant_along_rows_shifts_lse_only():
+    sq, sk, d = 7, 10, 4
+    q, k, v = _rand((sq, d), 1), _rand((sk, d), 2), _rand((sk, d), 3)
+    shift = _rand((sq, 1), 4)
+    o, lse = ref.forward(q, k, v, 0.5, INF, INF)
+    ob, lseb = ref.forward(q, k, v, 0.5, INF, INF, bias=np.broadcast_to(shift, (sq, sk)))
+    np.testing.assert_allclose(ob, o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lseb, lse + shift[:, 0], rtol=1e-13)
+    oz, lsez = ref.forward(q, k, v, 0.5, 2, 1, True, bias=np.zeros((sq, sk)))
+    o2, lse2 = ref.forward(q, k, v, 0.5, 2, 1, True)
+    np.testing.assert_array_equal(oz, o2)
+    np.testing.assert_array_equal(lsez, lse2)
+
+
+def test_planted_bias_inside_the_scale_is_caught():
+    # a slip that adds the bias before the scale, c (qk + B), fails the brute force
+    sq, sk, d = 4, 6, 3
+    q, k, v, do = (_rand(s, 95 + i) for i, s in enumerate([(sq, d), (sk, d), (sk, d), (sq, d)]))
+    bias = _rand((sq, sk), 99)
+    c = 0.4
+    mask = ref.allowed(sq, sk, INF, INF, False)
+    bad = ref._probs_block(q, k, c, mask, c * bias)[0] @ v   # c (qk + B)
+    bo = _brute_bias(q, k, v, do, c, (INF, INF, False), bias)[0]
+    assert not np.allclose(bad, bo, atol=1e-6)
