@@ -85,28 +85,31 @@ def _scale(p):
     return 0.0 if p >= 1.0 else 1.0 / (1.0 - p)
 
 
-def forward(q, k, v, sm_scale, window_left, window_right, bottom_right, p, seed, offset, bh):
-    """One (sequence, head) with dropout -> (O, LSE); LSE without dropout."""
+def forward(q, k, v, sm_scale, window_left, window_right, bottom_right, p, seed, offset, bh,
+            bias=None):
+    """One (sequence, head) with dropout -> (O, LSE); LSE without dropout.
+    ``bias`` [Sq, Sk] (optional) is added to the scaled scores."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     sq, sk = q.shape[0], k.shape[0]
     mask = ref.allowed(sq, sk, window_left, window_right, bottom_right)
-    probs, lse = ref._probs_block(q, k, sm_scale, mask)
+    probs, lse = ref._probs_block(q, k, sm_scale, mask, bias)
     m = keep_mask(seed, offset, bh, np.arange(sq), sk, p)
     return (probs * m * _scale(p)) @ v, lse
 
 
 def backward(q, k, v, do, sm_scale, window_left, window_right, bottom_right, p, seed, offset,
-             bh):
-    """One (sequence, head) with dropout: gradient of <dO, O> -> (dQ, dK, dV)."""
+             bh, bias=None):
+    """One (sequence, head) with dropout: gradient of <dO, O> -> (dQ, dK, dV),
+    or (dQ, dK, dV, dBias) with a ``bias`` (dBias = dS)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     do = np.asarray(do, dtype=np.float64)
     sq, sk = q.shape[0], k.shape[0]
     mask = ref.allowed(sq, sk, window_left, window_right, bottom_right)
-    probs, _ = ref._probs_block(q, k, sm_scale, mask)
+    probs, _ = ref._probs_block(q, k, sm_scale, mask, bias)
     ms = keep_mask(seed, offset, bh, np.arange(sq), sk, p) * _scale(p)
     pd = probs * ms
     o = pd @ v
@@ -114,4 +117,6 @@ def backward(q, k, v, do, sm_scale, window_left, window_right, bottom_right, p, 
     dp = (do @ v.T) * ms
     dlt = ref.delta(o, do)
     ds = probs * (dp - dlt[:, None])
+    if bias is not None:
+        return sm_scale * (ds @ k), sm_scale * (ds.T @ q), dv, ds
     return sm_scale * (ds @ k), sm_scale * (ds.T @ q), dv

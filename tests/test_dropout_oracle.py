@@ -136,3 +136,34 @@ def test_dropout_is_unbiased_over_masks():
     err = np.abs(samples.mean(0) - eo)
     se = samples.std(0, ddof=1) / np.sqrt(len(samples))
     assert (err <= 6 * se + 1e-12).all(), (err / (se + 1e-30)).max()
+
+
+@pytest.mark.parametrize("w", WINDOWS[:3], ids=str)
+def test_bias_with_dropout_p_zero_equals_the_bias_oracle(w):
+    q, k, v, do = _inputs(6, 9, 4, 6)
+    bias = 1.5 * np.random.default_rng(7).standard_normal((6, 9))
+    o, lse = dr.forward(q, k, v, 0.4, *w, 0.0, 5, 0, 0, bias=bias)
+    eo, el = ref.forward(q, k, v, 0.4, *w, bias=bias)
+    np.testing.assert_array_equal(o, eo)
+    np.testing.assert_array_equal(lse, el)
+    for g, e in zip(dr.backward(q, k, v, do, 0.4, *w, 0.0, 5, 0, 0, bias=bias),
+                    ref.backward(q, k, v, do, 0.4, *w, bias=bias)):
+        np.testing.assert_allclose(g, e, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("w", WINDOWS[:2], ids=str)
+def test_bias_gradient_under_dropout_matches_central_differences(w):
+    q, k, v, do = _inputs(5, 7, 3, 9)
+    bias = np.sin(np.arange(35, dtype=np.float64).reshape(5, 7))
+    args = (0.7, *w, 0.3, 1234, 9, 4)
+    *_, db = dr.backward(q, k, v, do, *args, bias=bias)
+    h = 1e-6
+    num = np.zeros_like(bias)
+    for pos in np.ndindex(bias.shape):
+        bp, bm = bias.copy(), bias.copy()
+        bp[pos] += h
+        bm[pos] -= h
+        lp = (dr.forward(q, k, v, *args, bias=bp)[0] * do).sum()
+        lm = (dr.forward(q, k, v, *args, bias=bm)[0] * do).sum()
+        num[pos] = (lp - lm) / (2 * h)
+    np.testing.assert_allclose(db, num, rtol=1e-5, atol=1e-7)
