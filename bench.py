@@ -232,10 +232,20 @@ def describe(w: synth.Workload):
                   f"{w.H * sum(sk) * w.D * 2 / 1e6:.0f} MB; L2 is 126 MB)"}
 
 
+def bias_bytes(w: synth.Workload, pairs: int):
+    """Algorithmic HBM bytes the additive bias adds (16-bit elements): the
+    forward reads B on the allowed pairs; the backward reads it there and
+    writes dB = dS over every (query, key) pair of each sequence (0 on the
+    masked ones)."""
+    sq, sk = seqlens(w)
+    every = w.H * sum(a * b for a, b in zip(sq, sk))
+    return {"attn_fwd_kernel": 2 * pairs, "attn_bwd_kernel": 2 * pairs + 2 * every}
+
+
 class Step:
     """Device buffers and the two C-ABI calls of one step."""
 
-    def __init__(self, w: synth.Workload, dev):
+    def __init__(self, w: synth.Workload, dev, bias: bool = False):
         from scaled_dot_product_12_b200 import binding as B
         self.B = B
         self.w = w
@@ -266,8 +276,17 @@ class Step:
         self.dq = torch.empty_like(self.q)
         self.dk = torch.empty_like(self.k)
         self.dv = torch.empty_like(self.v)
+        self.bias = self.dbias = None
+        if bias:
+            # [B, H, Sq, Sk] (largest lengths for packed inputs), drawn on the
+            # device: N(0, 1) from a seeded device generator
+            shape = (pr.B, w.H, pr.Sq, pr.Sk)
+            g = torch.Generator(device=dev).manual_seed(w.seed + 1)
+            self.bias = torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(dtype)
+            self.dbias = torch.empty_like(self.bias)
+            self.kw["bias"] = self.bias
         self.bp = B.bwd_params(self.do, self.q, self.k, self.v, self.o, self.lse, pr, self.dq,
-                               self.dk, self.dv)
+                               self.dk, self.dv, bias=self.bias, dbias=self.dbias)
         self.ws = torch.empty(max(1, B.workspace_bytes(self.bp)), dtype=torch.uint8, device=dev)
         self.bp.workspace = self.ws.data_ptr()
         self.bp.workspace_bytes = self.ws.numel()
@@ -310,10 +329,13 @@ def run_gpu(args, rank, world, local):
     w = synth.ALL_WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    step = Step(w, dev)
+    step = Step(w, dev, bias=args.bias)
     stream = torch.cuda.Stream(dev)
     fwd_flops, bwd_flops, pairs = workload_flops(w)
     nbytes = workload_bytes(w)
+    if args.bias:
+        for kname, extra in bias_bytes(w, pairs).items():
+            nbytes[kname] += extra
     flops = fwd_flops + bwd_flops
     peaks, peak_src = load_peaks()
 
@@ -372,7 +394,11 @@ def run_gpu(args, rank, world, local):
     roof["traffic"] = load_traffic(roof["kernel"], w.name)
 
     # ---- end to end through the C ABI with host buffers ----
-    e2e = run_e2e(step, stream, dev, min(args.steps, 5), flops, world)
+    if args.bias:
+        e2e = {"skipped": "bias runs measure the kernels only (the bias and its gradient "
+                          "would add two Sq x Sk tensors per head to every copy)"}
+    else:
+        e2e = run_e2e(step, stream, dev, min(args.steps, 5), flops, world)
 
     def per_kernel(tf, ms, nb):
         return {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4),
@@ -385,7 +411,9 @@ def run_gpu(args, rank, world, local):
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
         "data": "synthetic: i.i.d. N(0,1) Q, K, V, dO from a fixed seed",
-        "config": describe(w),
+        "config": dict(describe(w), **({"bias": "additive bias [B, H, Sq, Sk] N(0, 1) in the "
+                                                "input dtype, and its gradient"}
+                                       if args.bias else {})),
         "fwd": per_kernel(fwd_tf, fwd_ms, nbytes["attn_fwd_kernel"]),
         "bwd_main": per_kernel(bwd_tf, main_ms, nbytes["attn_bwd_kernel"]),
         "bwd_other_ms": round(ms_step - fwd_ms - main_ms, 4),
@@ -402,7 +430,7 @@ def run_gpu(args, rank, world, local):
         "e2e": e2e,
         "allowed_pairs": pairs,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.bias:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
 
@@ -668,6 +696,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="ltx_15300", choices=sorted(synth.ALL_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bias", action="store_true",
+                    help="add an additive bias [B, H, Sq, Sk] to the step and write its gradient "
+                         "(kernels only: no end-to-end or CPU leg)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

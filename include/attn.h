@@ -4,11 +4,12 @@
  *
  * What the calls compute.  For every sequence b and head h, with
  * c = sm_scale and the window of the sequence (below):
- *     S_ij = c * <q_i, k_j>,  LSE_i = ln sum_{allowed j} exp(S_ij),
+ *     S_ij = c * <q_i, k_j> (+ bias_ij, optional),  LSE_i = ln sum_{allowed j} exp(S_ij),
  *     P_ij = exp(S_ij - LSE_i) on allowed j (0 elsewhere),  O_i = sum_j P_ij v_j.
  * A row with no allowed key gets O_i = 0 and LSE_i = -inf.  attn_bwd returns
- * the gradient of <dO, O> with respect to Q, K and V:
- *     dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),  dQ = c dS K,  dK = c dS^T Q.
+ * the gradient of <dO, O> with respect to Q, K and V (and the bias):
+ *     dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),  dQ = c dS K,  dK = c dS^T Q,
+ *     dbias = dS.
  * The aotriton README (section "Kernel Support") names this kernel family:
  * FlashAttention after Tri Dao, which reaches the plain definition above.
  *
@@ -82,10 +83,11 @@ extern "C" {
 #endif
 
 /* Version 2 adds the fields after cu_seqlens_k (forward) / main_kernel_events
- * (backward).  A caller built against version 1 passes version 1 and the
- * version-1 struct size (ATTN_FWD_PARAMS_V1_SIZE / ATTN_BWD_PARAMS_V1_SIZE);
- * the version-2 fields then read as zero. */
-#define ATTN_PARAMS_VERSION 2u
+ * (backward), version 3 the bias fields after flags.  A caller built against
+ * an older version passes that version and its struct size
+ * (ATTN_FWD_PARAMS_V1_SIZE, ATTN_FWD_PARAMS_V2_SIZE and the backward
+ * counterparts); the fields it does not know then read as zero. */
+#define ATTN_PARAMS_VERSION 3u
 
 /* Return codes (numeric values of cudaError_t). */
 #define ATTN_SUCCESS 0
@@ -157,7 +159,8 @@ extern "C" {
  * Forward parameters.  Sizes: dense -- B batches of Sq queries and Sk keys;
  * packed -- B sequences, Sq / Sk the largest seqlen_q / seqlen_k (they size
  * the launch; a sequence longer than them is an error of the caller, whose
- * rows past Sq / Sk are left unwritten), total_q / total_k the rows of the
+ * results are then unspecified, though nothing outside the tensors, the
+ * bias included, is read or written), total_q / total_k the rows of the
  * packed tensors, cu_seqlens_q / _k device arrays of B + 1 int32 cumulative
  * lengths starting at 0 (each entry is clamped to [0, total_q] / [0,
  * total_k] on the device, so an array that runs past the tensors shortens
@@ -177,6 +180,19 @@ extern "C" {
  * philox_seed) is below floor((1 - dropout_p) * 2^32); kept elements are
  * scaled by 1 / (1 - dropout_p).  LSE is that of the softmax without
  * dropout.  The backward regenerates the same mask from the same fields.
+ *
+ * Additive bias (version 3; AOTriton 0.10b release notes, "Known Problems",
+ * and 0.14b notes, "Kernel Bug Fixes", where the bias is converted to fp32
+ * before it is added): with bias != NULL the logits are
+ *     S_ij = c * <q_i, k_j> + bias(b, h, i, j)
+ * on allowed pairs (the bias never unmasks a pair), with LSE, P and O taken
+ * from these S.  bias has the dtype of Q; element (b, h, i, j), i and j
+ * counted within sequence b (i < seqlen_q <= Sq, j < seqlen_k <= Sk), is at
+ * bias + b*bias_stride[0] + h*bias_stride[1] + i*bias_stride[2] + j in every
+ * varlen mode (a [B, H, Sq, Sk] tensor; elements past a sequence's lengths
+ * are not read).  bias_stride[0] and [1] may be 0 (one bias for all batches
+ * or heads); every stride's byte size is a multiple of 16 and the base is
+ * 16-byte aligned.  Bias entries must be finite.
  */
 typedef struct attn_fwd_params {
   uint32_t struct_size; /* sizeof(attn_fwd_params) */
@@ -203,8 +219,12 @@ typedef struct attn_fwd_params {
   uint64_t philox_seed;
   uint32_t philox_offset;
   uint32_t flags;              /* none defined for the forward: must be 0 */
+  /* ---- version 3 ---- */
+  const void* bias;            /* NULL: no bias */
+  int64_t bias_stride[3];      /* batch, head, query row (elements) */
 } attn_fwd_params;
 #define ATTN_FWD_PARAMS_V1_SIZE ((uint32_t)offsetof(attn_fwd_params, seqused_q))
+#define ATTN_FWD_PARAMS_V2_SIZE ((uint32_t)offsetof(attn_fwd_params, bias))
 
 /*
  * Backward parameters: the forward's fields plus the forward output O, its
@@ -215,6 +235,15 @@ typedef struct attn_fwd_params {
  * delta = rowsum(dO o O) [H][rows] followed by the fp32 dQ accumulator
  * [H][rows][D], rows = B*Sq (dense) or total_q (packed), and with
  * ATTN_BWD_DETERMINISTIC the int32 order counters [H][rows][4].
+ *
+ * Bias (version 3): the forward's bias (same fields, required to recompute
+ * P when the forward had one) and an optional output dbias, the gradient of
+ * <dO, O> with respect to the bias: dbias(b, h, i, j) = dS_ij on allowed
+ * pairs, 0 on masked pairs of the sequence, in the dtype of Q and addressed
+ * like the bias through dbias_stride (all of them positive where the extent
+ * is above 1: one element per (b, h, i, j); a caller that broadcast the bias
+ * sums the result itself).  Elements past a sequence's lengths are not
+ * written.  dbias without bias is the gradient at a zero bias.
  */
 typedef struct attn_bwd_params {
   uint32_t struct_size; /* sizeof(attn_bwd_params) */
@@ -252,8 +281,13 @@ typedef struct attn_bwd_params {
   uint64_t philox_seed;
   uint32_t philox_offset;
   uint32_t flags;              /* ATTN_BWD_DETERMINISTIC or 0 */
+  /* ---- version 3 ---- */
+  const void* bias;            /* the forward's bias, or NULL */
+  void* dbias;                 /* written when not NULL */
+  int64_t bias_stride[3], dbias_stride[3];
 } attn_bwd_params;
 #define ATTN_BWD_PARAMS_V1_SIZE ((uint32_t)offsetof(attn_bwd_params, seqused_q))
+#define ATTN_BWD_PARAMS_V2_SIZE ((uint32_t)offsetof(attn_bwd_params, bias))
 
 /* attn_bwd_params.flags: add the dQ contributions of the key tiles in a
  * fixed order, so that repeated calls give bit-identical dQ (AOTriton 0.15b
@@ -285,6 +319,9 @@ ATTN_API size_t attn_bwd_workspace_size(const attn_bwd_params* params);
  * bytes, which every GPU that loads the library holds until the process exits.
  * The caller passes inputs and outputs only; params->workspace and
  * params->workspace_bytes are ignored.  The call allocates nothing.
+ *   - params must be of the current version (struct_size ==
+ *     sizeof(attn_bwd_params)); older struct sizes are rejected with
+ *     ATTN_ERROR_INVALID_VALUE.
  *   - Sizes whose attn_bwd_workspace_size() exceeds ATTN_STATIC_WORKSPACE_BYTES
  *     are rejected with cudaErrorMemoryAllocation (2) before any GPU work;
  *     otherwise the return codes are those of attn_bwd.

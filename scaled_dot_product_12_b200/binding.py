@@ -19,7 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libattn.so")
 
 # Constants of include/attn.h
-PARAMS_VERSION = 2
+PARAMS_VERSION = 3
 BWD_DETERMINISTIC = 1
 DTYPE_FP16, DTYPE_BF16 = 0, 1
 WINDOW_INF = 2**31 - 1
@@ -66,6 +66,8 @@ class FwdParams(ctypes.Structure):
         ("seqused_q", ctypes.c_void_p), ("seqused_k", ctypes.c_void_p), ("Dv", ctypes.c_int32),
         ("dropout_p", ctypes.c_float), ("philox_seed", ctypes.c_uint64),
         ("philox_offset", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+        # version 3
+        ("bias", ctypes.c_void_p), ("bias_stride", _i64x3),
     ]
 
 
@@ -88,12 +90,18 @@ class BwdParams(ctypes.Structure):
         ("seqused_q", ctypes.c_void_p), ("seqused_k", ctypes.c_void_p), ("Dv", ctypes.c_int32),
         ("dropout_p", ctypes.c_float), ("philox_seed", ctypes.c_uint64),
         ("philox_offset", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+        # version 3
+        ("bias", ctypes.c_void_p), ("dbias", ctypes.c_void_p),
+        ("bias_stride", _i64x3), ("dbias_stride", _i64x3),
     ]
 
 
-# Size of the version-1 structs (every field before seqused_q).
+# Sizes of the older structs: version 1 ends before seqused_q, version 2
+# before bias.
 FWD_PARAMS_V1_SIZE = FwdParams.seqused_q.offset
 BWD_PARAMS_V1_SIZE = BwdParams.seqused_q.offset
+FWD_PARAMS_V2_SIZE = FwdParams.bias.offset
+BWD_PARAMS_V2_SIZE = BwdParams.bias.offset
 
 
 EXPORTS = {
@@ -265,12 +273,28 @@ class Problem:
         p.flags = self.flags
 
 
+def _bias_strides(t: Optional[torch.Tensor], q: torch.Tensor, name: str):
+    """Strides of a [B, H, Sq, Sk] bias (or its gradient), checked for shape
+    rank, dtype and a contiguous key dimension; the library checks the rest."""
+    if t is None:
+        return _i64x3(0, 0, 0)
+    if t.dim() != 4:
+        raise ValueError(f"{name}: a [B, H, Sq, Sk] tensor is expected")
+    if t.dtype != q.dtype:
+        raise ValueError(f"{name}: dtype {t.dtype} differs from q's {q.dtype}")
+    if t.shape[3] > 1 and t.stride(3) != 1:
+        raise ValueError(f"{name}: the key dimension must be contiguous")
+    s = t.stride()
+    return _i64x3(s[0] if t.shape[0] > 1 else 0, s[1] if t.shape[1] > 1 else 0,
+                  s[2] if t.shape[2] > 1 else 0)
+
+
 def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_right=False,
             cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None,
             lse_layout="HT", out=None, lse=None, return_lse=True, stream=None,
             seqlens_q=None, seqlens_k=None, seqused_q=None, seqused_k=None, seqstart_q=None,
             seqstart_k=None, dropout_p=0.0, philox_seed=0,
-            philox_offset=0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            philox_offset=0, bias=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """O (and LSE) of FlashAttention through attn_fwd.
 
     Dense: q [B,H,Sq,D], k/v [B,H,Sk,D].  Packed: q [Tq,H,D], k/v [Tk,H,D] with
@@ -280,6 +304,9 @@ def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_righ
     packed tensor.  Padded: dense shapes plus int32 seqlens_q / seqlens_k [B]
     on the device.  Rows outside every sequence are left untouched.  dropout_p
     > 0 drops elements of P with the Philox generator keyed by philox_seed.
+    ``bias`` [B, H, Sq, Sk] (q's dtype; batch and head may be broadcast with
+    ``expand``) is added to the scaled scores, (i, j) counted within each
+    sequence.
     """
     pr = Problem(q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
                  max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k, seqused_q,
@@ -297,11 +324,13 @@ def forward(q, k, v, sm_scale=None, window=(WINDOW_INF, WINDOW_INF), bottom_righ
     p.k_stride = _strides(k, pr.k_packed)
     p.v_stride = _strides(v, pr.k_packed)
     p.o_stride = _strides(out, pr.q_packed)
+    p.bias, p.bias_stride = _ptr(bias), _bias_strides(bias, q, "bias")
     _check("attn_fwd", lib().attn_fwd(ctypes.byref(p), _stream_handle(q.device, stream)))
     return out, lse
 
 
-def bwd_params(dout, q, k, v, o, lse, pr: Problem, dq, dk, dv, workspace=None) -> BwdParams:
+def bwd_params(dout, q, k, v, o, lse, pr: Problem, dq, dk, dv, workspace=None, bias=None,
+               dbias=None) -> BwdParams:
     p = BwdParams()
     pr.fill(p, _dtype_code(q))
     p.q, p.k, p.v, p.o, p.dout, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse)
@@ -311,6 +340,8 @@ def bwd_params(dout, q, k, v, o, lse, pr: Problem, dq, dk, dv, workspace=None) -
                     ("dv", dv)):
         setattr(p, name + "_stride", _strides(t, pr.k_packed if name in ("k", "v", "dk", "dv")
                                               else pr.q_packed))
+    p.bias, p.bias_stride = _ptr(bias), _bias_strides(bias, q, "bias")
+    p.dbias, p.dbias_stride = _ptr(dbias), _bias_strides(dbias, q, "dbias")
     if workspace is not None:
         p.workspace = workspace.data_ptr()
         p.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -326,9 +357,11 @@ def backward(dout, q, k, v, o, lse, sm_scale=None, window=(WINDOW_INF, WINDOW_IN
              max_seqlen_k=None, lse_layout="HT", dq=None, dk=None, dv=None, workspace=None,
              stream=None, seqlens_q=None, seqlens_k=None, seqused_q=None, seqused_k=None,
              seqstart_q=None, seqstart_k=None, dropout_p=0.0, philox_seed=0, philox_offset=0,
-             deterministic=False):
+             deterministic=False, bias=None, dbias=None):
     """(dQ, dK, dV) through attn_bwd; the workspace is allocated if not given.
-    ``deterministic`` adds the dQ contributions in a fixed order."""
+    ``deterministic`` adds the dQ contributions in a fixed order.  ``bias`` is
+    the forward's bias; ``dbias`` (a [B, H, Sq, Sk] tensor, not broadcast)
+    receives the gradient with respect to the bias."""
     pr = Problem(q, k, sm_scale, window, bottom_right, cu_seqlens_q, cu_seqlens_k,
                  max_seqlen_q, max_seqlen_k, lse_layout, seqlens_q, seqlens_k, seqused_q,
                  seqused_k, seqstart_q, seqstart_k)
@@ -337,7 +370,7 @@ def backward(dout, q, k, v, o, lse, sm_scale=None, window=(WINDOW_INF, WINDOW_IN
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    p = bwd_params(dout, q, k, v, o, lse, pr, dq, dk, dv)
+    p = bwd_params(dout, q, k, v, o, lse, pr, dq, dk, dv, bias=bias, dbias=dbias)
     need = workspace_bytes(p)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)

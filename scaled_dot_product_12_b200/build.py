@@ -49,18 +49,24 @@ def nvcc() -> str:
 
 
 def build(verbose: bool = False, extra_flags=()) -> str:
-    """Compile every source to an object, then link the shared library."""
+    """Compile every source to an object (in parallel), then link the shared
+    library."""
     out_dir = os.path.join(ROOT, "_build")
     os.makedirs(out_dir, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in SOURCES:
         obj = os.path.join(out_dir, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", os.path.join(ROOT, "include"),
-               "-c", os.path.join(CSRC, src), "-o", obj]
+        cmds.append([nvcc(), *NVCC_FLAGS, *extra_flags, "-I", os.path.join(ROOT, "include"),
+                     "-c", os.path.join(CSRC, src), "-o", obj])
+        objs.append(obj)
+    procs = []
+    for cmd in cmds:
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        procs.append((cmd, subprocess.Popen(cmd)))
+    failed = [cmd for cmd, pr in procs if pr.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
     tmp = library_path() + ".tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
            "-Xcompiler", "-fPIC", *objs, "-o", tmp]

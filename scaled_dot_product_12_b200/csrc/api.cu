@@ -142,18 +142,19 @@ bool decode_bits(uint32_t bits, Mode* m) {
   return true;
 }
 
-// Copies a version-1 or version-2 params struct into a full version-2 one
-// (version-1 callers get zeros in the fields they do not know).
+// Copies a params struct of any version into a full current one (callers of
+// an older version get zeros in the fields they do not know).
 template <class P>
-bool normalize(const P* in, uint32_t v1_size, P* out) {
+bool normalize(const P* in, uint32_t v1_size, uint32_t v2_size, P* out) {
   if (!in) return false;
   if (in->version == ATTN_PARAMS_VERSION && in->struct_size == sizeof(P)) {
     std::memcpy(out, in, sizeof(P));
     return true;
   }
-  if (in->version == 1u && in->struct_size == v1_size) {
+  const uint32_t known = in->version == 1u ? v1_size : in->version == 2u ? v2_size : 0u;
+  if (known != 0u && in->struct_size == known) {
     std::memset(out, 0, sizeof(P));
-    std::memcpy(out, in, v1_size);
+    std::memcpy(out, in, known);
     out->struct_size = sizeof(P);
     out->version = ATTN_PARAMS_VERSION;
     return true;
@@ -174,6 +175,19 @@ bool strides_ok(const int64_t* st, bool packed, int64_t nb, int64_t nh, int64_t 
   };
   if (!packed && !ok(st[0], nb)) return false;
   return ok(st[1], nh) && ok(st[2], nrows);
+}
+
+// Strides (elements) of a [B, H, Sq, Sk] bias: byte sizes multiples of 16,
+// batch and head strides may be 0 (broadcast) when `broadcast` allows it,
+// the row stride positive where there is more than one row.
+bool bias_strides_ok(const int64_t* st, int64_t nb, int64_t nh, int64_t nrows, bool broadcast) {
+  const int64_t lim = (int64_t)1 << 38;
+  auto ok = [&](int64_t s, int64_t extent, bool zero_ok) {
+    if (extent <= 1) return true;
+    if (s == 0) return zero_ok;
+    return s > 0 && s < lim && ((s * 2) % 16) == 0;
+  };
+  return ok(st[0], nb, broadcast) && ok(st[1], nh, broadcast) && ok(st[2], nrows, false);
 }
 
 cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, int H, int B,
@@ -263,7 +277,7 @@ extern "C" {
 
 int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
   attn_fwd_params full;
-  if (!normalize(params, ATTN_FWD_PARAMS_V1_SIZE, &full)) return cudaErrorInvalidValue;
+  if (!normalize(params, ATTN_FWD_PARAMS_V1_SIZE, ATTN_FWD_PARAMS_V2_SIZE, &full)) return cudaErrorInvalidValue;
   const attn_fwd_params* p = &full;
   Mode m;
   if (!common_ok(p, &m, /*known_flags=*/0u)) return cudaErrorInvalidValue;
@@ -280,6 +294,8 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
       !strides_ok(p->o_stride, m.q_packed, p->B, p->H, nq) ||
       !strides_ok(p->k_stride, m.k_packed, p->B, p->H, nk) ||
       !strides_ok(p->v_stride, m.k_packed, p->B, p->H, nk))
+    return cudaErrorInvalidValue;
+  if (p->bias && (!aligned16(p->bias) || !bias_strides_ok(p->bias_stride, p->B, p->H, p->Sq, true)))
     return cudaErrorInvalidValue;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
@@ -331,6 +347,8 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
     a.dev = dev;
     a.sms = info.sms;
     set_dropout(a, p);
+    a.bias = p->bias;
+    for (int i = 0; i < 3; ++i) a.bias_stride[i] = p->bias_stride[i];
     return attn::launch_fwd(a, stream);
   });
 }
@@ -358,7 +376,7 @@ constexpr bool kBwdDropout = true;                       // backward dropout ker
 
 size_t attn_bwd_workspace_size(const attn_bwd_params* params) {
   attn_bwd_params full;
-  if (!normalize(params, ATTN_BWD_PARAMS_V1_SIZE, &full)) return 0;
+  if (!normalize(params, ATTN_BWD_PARAMS_V1_SIZE, ATTN_BWD_PARAMS_V2_SIZE, &full)) return 0;
   Mode m;
   if (!common_ok(&full, &m, kBwdFlags, /*check_pointers=*/false, kBwdDropout)) return 0;
   return bwd_workspace(&full, m).total();
@@ -366,7 +384,7 @@ size_t attn_bwd_workspace_size(const attn_bwd_params* params) {
 
 int attn_bwd(const attn_bwd_params* params, void* stream_ptr) {
   attn_bwd_params full;
-  if (!normalize(params, ATTN_BWD_PARAMS_V1_SIZE, &full)) return cudaErrorInvalidValue;
+  if (!normalize(params, ATTN_BWD_PARAMS_V1_SIZE, ATTN_BWD_PARAMS_V2_SIZE, &full)) return cudaErrorInvalidValue;
   const attn_bwd_params* p = &full;
   Mode m;
   if (!common_ok(p, &m, kBwdFlags, true, kBwdDropout)) return cudaErrorInvalidValue;
@@ -396,6 +414,11 @@ int attn_bwd(const attn_bwd_params* params, void* stream_ptr) {
   const int64_t* sk_list[] = {p->k_stride, p->v_stride, p->dk_stride, p->dv_stride};
   for (const int64_t* st : sk_list)
     if (!strides_ok(st, m.k_packed, p->B, p->H, nk)) return cudaErrorInvalidValue;
+  if (p->bias && (!aligned16(p->bias) || !bias_strides_ok(p->bias_stride, p->B, p->H, p->Sq, true)))
+    return cudaErrorInvalidValue;
+  if (p->dbias &&
+      (!aligned16(p->dbias) || !bias_strides_ok(p->dbias_stride, p->B, p->H, p->Sq, false)))
+    return cudaErrorInvalidValue;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   return on_stream_device(stream, [&](int dev, const DeviceInfo& info) -> cudaError_t {
@@ -471,6 +494,12 @@ int attn_bwd(const attn_bwd_params* params, void* stream_ptr) {
     a.dev = dev;
     a.sms = info.sms;
     set_dropout(a, p);
+    a.bias = p->bias;
+    a.dbias = p->dbias;
+    for (int i = 0; i < 3; ++i) {
+      a.bias_stride[i] = p->bias_stride[i];
+      a.dbias_stride[i] = p->dbias_stride[i];
+    }
     a.main_events[0] = static_cast<cudaEvent_t>(p->main_kernel_events[0]);
     a.main_events[1] = static_cast<cudaEvent_t>(p->main_kernel_events[1]);
     return attn::launch_bwd(a, stream);

@@ -25,6 +25,8 @@
 // registers go to the others through setmaxnreg).
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "fwd.h"
 #include "mask.cuh"
@@ -261,7 +263,7 @@ __device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t
   }
 }
 
-template <int DPAD, bool BF16, bool DROPOUT>
+template <int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<DPAD>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -304,13 +306,42 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     return reinterpret_cast<uint8_t*>(base) + 2 * off;
   };
 
+  // dbias rows [r_begin, r_end) of this key tile's columns (those below
+  // seqlen_k) set to 0: the query rows no visited query tile holds, whose
+  // pairs with these keys are all masked.  Threads t of nt share the rows,
+  // 16 per row.
+  auto zero_dbias_rows = [&](int32_t r_begin, int32_t r_end, int t, int nt) {
+    if constexpr (BIAS) {
+      if (!a.dbias) return;
+      // (never past the bias tensor's Sq x Sk, whatever the sequence lengths)
+      const int ncols = min(128, min(sk, a.Sk) - n0);
+      r_end = min(r_end, a.Sq);
+      uint16_t* base = reinterpret_cast<uint16_t*>(a.dbias) + (int64_t)b * a.dbias_stride[0] +
+                       (int64_t)h * a.dbias_stride[1] + n0;
+      for (int64_t x = t; x < (int64_t)(r_end - r_begin) * 16; x += nt) {
+        const int32_t i = r_begin + (int32_t)(x >> 4);
+        const int c = (int)(x & 15);
+        if (8 * c >= ncols) continue;
+        uint16_t* p = base + (int64_t)i * a.dbias_stride[2] + 8 * c;
+        if (8 * c + 8 <= ncols) {
+          st_global_v4(p, 0u, 0u, 0u, 0u);
+        } else {
+          for (int e = 0; e < ncols - 8 * c; ++e) p[e] = 0;
+        }
+      }
+    } else {
+      (void)r_begin, (void)r_end, (void)t, (void)nt;
+    }
+  };
+
   if (n_it <= 0) {
-    // No query sees these keys: dK = dV = 0.
+    // No query sees these keys: dK = dV = 0 (and dbias = 0 in their columns).
     const int rows = min(128, sk - n0);
     for (int r = threadIdx.x / 4; r < rows; r += blockDim.x / 4) {
       zero_row16(kv_row_ptr(a.dk, a.dk_stride, n0 + r), a.D, threadIdx.x & 3, 4);
       zero_row16(kv_row_ptr(a.dv, a.dv_stride, n0 + r), a.Dv, threadIdx.x & 3, 4);
     }
+    zero_dbias_rows(0, sq, threadIdx.x, blockDim.x);
     return;
   }
 
@@ -530,6 +561,11 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       else
         issue_all(Flag<false>{});
     }
+  } else if (BIAS) {
+    // Warps 14-15: dbias of the query rows outside the visited tiles.
+    const int t = (warp - 14) * 32 + lane;
+    zero_dbias_rows(0, min(mb * 128, sq), t, 64);
+    zero_dbias_rows(min(me * 128, sq), sq, t, 64);
   }
   } else if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kPdsRegs));
@@ -548,6 +584,20 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     if (qa < 0) qa = 0;
     if (qz > sq - 1) qz = sq - 1;
     if (j >= sk) qz = qa - 1;
+    // Bias and dbias columns of key j (null past the sequence, or when not
+    // given): element (i, j) at col + i * stride.
+    const uint16_t* bcol = nullptr;
+    uint16_t* dbcol = nullptr;
+    const int32_t sqb = min(sq, a.Sq);  // bias rows: never past the tensor's Sq
+    (void)sqb;
+    if constexpr (BIAS) {
+      if (j < sk && j < a.Sk && a.bias)
+        bcol = reinterpret_cast<const uint16_t*>(a.bias) + (int64_t)b * a.bias_stride[0] +
+               (int64_t)h * a.bias_stride[1] + j;
+      if (j < sk && j < a.Sk && a.dbias)
+        dbcol = reinterpret_cast<uint16_t*>(a.dbias) + (int64_t)b * a.dbias_stride[0] +
+                (int64_t)h * a.dbias_stride[1] + j;
+    }
     // Per-query values of a tile, one per thread: group 0 fetches LSE, group
     // 1 fetches delta, for query row r (0 past the sequence).
     auto row_val = [&](int it) -> float {
@@ -663,17 +713,44 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       uint32_t pk[32];
       uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
       if constexpr (DROPOUT) stage_delta(it);
+      if constexpr (BIAS) {
+        // the next tile's bias column into L2 (rows qo .. qo + 63 of it)
+        if (bcol && it + 1 < n_it) {
+          const int32_t i1 = m0 + 128 + qo;
+          const int nr = min(64, sqb - i1);
+          const uint16_t* p = bcol + (int64_t)i1 * a.bias_stride[2];
+          for (int k = lane & 1; k < nr; k += 2)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (int64_t)k * a.bias_stride[2]));
+        }
+      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         if constexpr (DROPOUT) keep[c] = keep_bits(it, c);
+        // bias(i, j) of the chunk's 32 queries, times log2(e); 0 past seqlen_q
+        float bl[BIAS ? 32 : 1];
+        if constexpr (BIAS) {
+          const int32_t i0 = m0 + qo + 32 * c;
+          const uint16_t* p = bcol ? bcol + (int64_t)i0 * a.bias_stride[2] : nullptr;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            bl[k] = (p && i0 + k < sqb)
+                        ? h16_to_f32<BF16>(__ldg(p + (int64_t)k * a.bias_stride[2])) * 1.4426950408889634f
+                        : 0.f;
+        }
         uint32_t sr[32];
         tmem_ld32(tS + qo + 32 * c, sr);
         uint32_t chunk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int q0 = qo + 32 * c + 2 * e, q1 = q0 + 1;
-          float v0 = ex2(__uint_as_float(sr[2 * e]) * sl2);
-          float v1 = ex2(__uint_as_float(sr[2 * e + 1]) * sl2);
+          float v0, v1;
+          if constexpr (BIAS) {
+            v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, bl[2 * e]));
+            v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, bl[2 * e + 1]));
+          } else {
+            v0 = ex2(__uint_as_float(sr[2 * e]) * sl2);
+            v1 = ex2(__uint_as_float(sr[2 * e + 1]) * sl2);
+          }
           if (!full) {
             v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
             v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
@@ -730,6 +807,15 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
             d1 = pe.y * __uint_as_float(dr[2 * e + 1]);
           }
           dd[e] = pack2<BF16>(d0, d1);
+          if constexpr (BIAS) {
+            // dbias(i, j) = dS (queries past seqlen_q are not written)
+            const int32_t i = m0 + qo + 32 * c + 2 * e;
+            if (dbcol && i < sqb) {
+              uint16_t* p = dbcol + (int64_t)i * a.dbias_stride[2];
+              p[0] = (uint16_t)(dd[e] & 0xFFFFu);
+              if (i + 1 < sqb) p[a.dbias_stride[2]] = (uint16_t)(dd[e] >> 16);
+            }
+          }
         }
         tmem_st16(tDP + po + 16 * c, dd);
         // dS (query-contiguous rows of this key) into the MN-major smem tile:
@@ -897,14 +983,14 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   }
 }
 
-template <int DPAD, bool BF16, bool DROPOUT>
+template <int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 static cudaError_t launch_main(const BwdArgs& a, cudaStream_t stream) {
   using C = BwdCfg<DPAD>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   // One warp of each warpgroup per sub-partition: P/dS, P/dS, drain, TMA/MMA.
   static_assert(2 * C::kPdsRegs + C::kDrainRegs + C::kProducerRegs <= 4 * C::kLaunchRegs,
                 "register split exceeds the launch budget");
-  auto kern = attn_bwd_kernel<DPAD, BF16, DROPOUT>;
+  auto kern = attn_bwd_kernel<DPAD, BF16, DROPOUT, BIAS>;
   static std::atomic<uint64_t> prepared{0};
   const dim3 grid((a.Sk + 127) / 128, a.H, a.B);
   return prepared_launch(kern, prepared, a.dev, C::kSmemBytes, C::kLaunchRegs, [&] {
@@ -927,10 +1013,17 @@ static cudaError_t launch_all(const BwdArgs& a, cudaStream_t stream, int sms) {
     if (a.main_events[0] && (e = cudaEventRecord(a.main_events[0], stream)) != cudaSuccess) return e;
     // all tiles take the wider of the two head dims (TMA zero-fills the rest)
     const bool narrow = a.D <= 64 && a.Dv <= 64;
-    if (a.dropout)
-      e = narrow ? launch_main<64, BF16, true>(a, stream) : launch_main<128, BF16, true>(a, stream);
-    else
-      e = narrow ? launch_main<64, BF16, false>(a, stream) : launch_main<128, BF16, false>(a, stream);
+    const bool bias = a.bias || a.dbias;
+    auto by_bias = [&](auto dpad, auto drop) -> cudaError_t {
+      constexpr int P = decltype(dpad)::value;
+      constexpr bool DR = decltype(drop)::value;
+      return bias ? launch_main<P, BF16, DR, true>(a, stream) : launch_main<P, BF16, DR, false>(a, stream);
+    };
+    auto by_drop = [&](auto dpad) -> cudaError_t {
+      return a.dropout ? by_bias(dpad, Flag<true>{}) : by_bias(dpad, Flag<false>{});
+    };
+    e = narrow ? by_drop(std::integral_constant<int, 64>{})
+               : by_drop(std::integral_constant<int, 128>{});
     if (e != cudaSuccess) return e;
     if (a.main_events[1] && (e = cudaEventRecord(a.main_events[1], stream)) != cudaSuccess) return e;
   }

@@ -465,6 +465,34 @@ __device__ __forceinline__ void zero_row16(uint8_t* row, int ncols, int t, int n
     *reinterpret_cast<uint16_t*>(row + 2 * col) = 0;
 }
 
+// Eight 16-bit values at p (16-byte aligned) as four packed pairs, only the
+// first `ncols` of them read (the others, and all of them when ncols <= 0,
+// are 0).  Read-only data: the non-coherent path.
+__device__ __forceinline__ uint4 ld_row8(const uint16_t* p, int ncols) {
+  if (ncols >= 8) return __ldg(reinterpret_cast<const uint4*>(p));
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (e < ncols) w[e >> 1] |= (uint32_t)__ldg(p + e) << (16 * (e & 1));
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+// A 16-bit value as fp32.
+template <bool BF16>
+__device__ __forceinline__ float h16_to_f32(uint32_t bits) {
+  if constexpr (BF16) {
+    return __uint_as_float(bits << 16);
+  } else {
+    return __half2float(__ushort_as_half((unsigned short)bits));
+  }
+}
+// L2 prefetch of the 128-byte lines that hold the first, the 65th and the
+// last of `ncols` (1..128) consecutive 16-bit values at p.
+__device__ __forceinline__ void prefetch_row_l2(const uint16_t* p, int ncols) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+  if (ncols > 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 64));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (ncols - 1)));
+}
+
 // A compile-time flag passed to generic lambdas (for `if constexpr` code
 // paths instantiated per call site).
 template <bool V>

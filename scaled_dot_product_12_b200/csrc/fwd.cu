@@ -27,6 +27,8 @@
 // [128 NQ + DPAD t, ...).
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "fwd.h"
 #include "mask.cuh"
@@ -176,7 +178,7 @@ __device__ __forceinline__ bool fwd_unit(const FwdArgs& a, int32_t n_mblocks, co
   return true;
 }
 
-template <int NQ, int DPAD, bool BF16, bool DROPOUT>
+template <int NQ, int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ FwdArgs args) {
   using C = FwdCfg<NQ, DPAD>;
@@ -484,19 +486,63 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       const int32_t lo = row_lo(w.win, i), hi = row_hi(w.win, i, w.sk);
       const uint32_t bh = (uint32_t)(w.b * args.H + w.h);  // dropout counter word
       (void)bh;
+      // Bias row of query i (null past the sequence, or past the bias
+      // tensor's Sq rows for an over-long sequence: those rows read 0).
+      const uint16_t* brow = nullptr;
+      if constexpr (BIAS) {
+        if (valid && i < args.Sq)
+          brow = reinterpret_cast<const uint16_t*>(args.bias) + (int64_t)w.b * args.bias_stride[0] +
+                 (int64_t)w.h * args.bias_stride[1] + (int64_t)i * args.bias_stride[2];
+      }
+      // With a bias the logits are formed in the log2 domain below
+      // (c S log2(e) + B log2(e)), and the shift works at unit scale.
+      const float sl2e = BIAS ? 1.f : sl2;
       float m_used = -INFINITY, l = 0.f;
       for (int it = 0; it < w.n_tiles; ++it) {
         const int64_t gi = g + it;
+        const int32_t n0 = (w.nb + it) * 128;
+        // The tile's bias (columns n0 .. n0 + 127, those past seqlen_k read
+        // as 0) is requested before the wait for S, and the next tile's
+        // lines are prefetched into L2.
+        uint4 bq[BIAS ? 16 : 1];
+        if constexpr (BIAS) {
+          const int32_t left = brow ? min(w.sk, args.Sk) - n0 : 0;
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            bq[q] = left > 8 * q ? ld_row8(brow + n0 + 8 * q, left - 8 * q) : make_uint4(0, 0, 0, 0);
+          if (brow && it + 1 < w.n_tiles && left > 128)
+            prefetch_row_l2(brow + n0 + 128, min(left - 128, 128));
+        }
         ok = mbar_wait(s_full(t), (uint32_t)(gi & 1), abort_flag, args.status, kSiteSoftmax);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        // The whole score row in one TMEM load.
-        uint32_t raw[128];
-        tmem_ld128(tS, raw);
         float s[128];
+        if constexpr (BIAS) {
+          // Four TMEM loads of 32 columns, each folded with its bias columns
+          // at once, so the raw scores and the bias are never all live.
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c]);
-        const int32_t n0 = (w.nb + it) * 128;
+          for (int part = 0; part < 4; ++part) {
+            uint32_t raw[32];
+            tmem_ld32(tS + 32 * part, raw);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = bq[4 * part + q];
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int c = 32 * part + 8 * q + e;
+                const float bias = h16_to_f32<BF16>((wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
+                s[c] = fmaf(__uint_as_float(raw[8 * q + e]), sl2, bias * 1.4426950408889634f);
+              }
+            }
+          }
+        } else {
+          // The whole score row in one TMEM load.
+          uint32_t raw[128];
+          tmem_ld128(tS, raw);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c]);
+        }
         const bool full = tile_is_full(w.win, w.sq, w.sk, w.m0 + 128 * t, n0);
         if (!full) {
           const int32_t a = lo - n0, z = hi - n0;  // allowed columns [a, z]
@@ -518,7 +564,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[120 + k]);
         const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
                                fmaxf(m8[6], m8[7]));
-        const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2;
+        const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2e;
         // Lazy rescale: keep the running reference unless the new maximum
         // exceeds it by more than 2^8 (P stays below 256, exact in fp32 sums).
         float alpha = 1.f;
@@ -529,7 +575,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
         const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
         // Scale-and-shift and the row sum run on packed fp32 pairs.
         uint64_t l4[4] = {0, 0, 0, 0};
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+        const uint64_t sl2x2 = f2_pack(sl2e, sl2e), negm2 = f2_pack(neg_m, neg_m);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           // Dropout: bit k of `keep` says whether column 32 c + k survives.
@@ -630,13 +676,13 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
   }
 }
 
-template <int NQ, int DPAD, bool BF16, bool DROPOUT>
+template <int NQ, int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 static cudaError_t launch(const FwdArgs& args, int64_t n_units, cudaStream_t stream) {
   using C = FwdCfg<NQ, DPAD>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   static_assert(NQ * 128 * C::kHighRegs + 128 * C::kLowRegs <= C::kThreads * C::kLaunchRegs,
                 "register split exceeds the launch budget");
-  auto kern = attn_fwd_kernel<NQ, DPAD, BF16, DROPOUT>;
+  auto kern = attn_fwd_kernel<NQ, DPAD, BF16, DROPOUT, BIAS>;
   static std::atomic<uint64_t> prepared{0};
   // One CTA per SM (the shared-memory footprint allows no second one).
   const int64_t sms = args.sms > 0 ? args.sms : 148;
@@ -655,18 +701,22 @@ cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream) {
   // Q, K, V and O tiles all take the wider of the two head dims (TMA fills
   // the columns past a tensor's own head dim with zeros).
   const bool narrow = args.D <= 64 && args.Dv <= 64;
-  if (args.dropout) {
-    if (narrow)
-      return bf16 ? launch<NQ, 64, true, true>(args, n_units, stream)
-                  : launch<NQ, 64, false, true>(args, n_units, stream);
-    return bf16 ? launch<NQ, 128, true, true>(args, n_units, stream)
-                : launch<NQ, 128, false, true>(args, n_units, stream);
-  }
-  if (narrow)
-    return bf16 ? launch<NQ, 64, true, false>(args, n_units, stream)
-                : launch<NQ, 64, false, false>(args, n_units, stream);
-  return bf16 ? launch<NQ, 128, true, false>(args, n_units, stream)
-              : launch<NQ, 128, false, false>(args, n_units, stream);
+  // Runtime choices to template arguments: head-dim class, dtype, dropout,
+  // bias.
+  auto by_bias = [&](auto dpad, auto bf, auto drop) -> cudaError_t {
+    constexpr int P = decltype(dpad)::value;
+    constexpr bool F = decltype(bf)::value, DR = decltype(drop)::value;
+    return args.bias ? launch<NQ, P, F, DR, true>(args, n_units, stream)
+                     : launch<NQ, P, F, DR, false>(args, n_units, stream);
+  };
+  auto by_drop = [&](auto dpad, auto bf) -> cudaError_t {
+    return args.dropout ? by_bias(dpad, bf, Flag<true>{}) : by_bias(dpad, bf, Flag<false>{});
+  };
+  auto by_dtype = [&](auto dpad) -> cudaError_t {
+    return bf16 ? by_drop(dpad, Flag<true>{}) : by_drop(dpad, Flag<false>{});
+  };
+  return narrow ? by_dtype(std::integral_constant<int, 64>{})
+                : by_dtype(std::integral_constant<int, 128>{});
 }
 
 }  // namespace attn

@@ -42,6 +42,10 @@ struct FwdArgs {
   int32_t dropout;
   uint32_t keep_below, seed_lo, seed_hi, philox_offset;
   float drop_scale;
+  // Additive bias: element (b, h, i, j) of sequence b at bias + b*s[0] +
+  // h*s[1] + i*s[2] + j (16-bit, the dtype of Q), or null.
+  const void* bias;
+  int64_t bias_stride[3];
 };
 
 struct BwdArgs {
@@ -79,6 +83,11 @@ struct BwdArgs {
   int32_t dropout;             // as in FwdArgs
   uint32_t keep_below, seed_lo, seed_hi, philox_offset;
   float drop_scale;
+  // Bias as in FwdArgs (null: zero) and its gradient dS, addressed the same
+  // way through dbias_stride (null: not written).
+  const void* bias;
+  void* dbias;
+  int64_t bias_stride[3], dbias_stride[3];
 };
 
 cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream);

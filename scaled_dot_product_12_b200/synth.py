@@ -46,6 +46,12 @@ def qkv_do(q_shape, k_shape, seed: int, dtype=torch.bfloat16, dv: Optional[int] 
     return q, k, v, do
 
 
+def bias(shape, seed: int, dtype=torch.bfloat16, std: float = 1.0):
+    """An additive attention bias: i.i.d. N(0, std^2) drawn in fp32 on the CPU
+    from its own generator, rounded to ``dtype``."""
+    return (normal(shape, seed, torch.float32) * std).to(dtype)
+
+
 def varlen_seqlens(seed: int, n_seqs: int = 16, max_q: int = 4096, max_extra_k: int = 512):
     """seqlen_q ~ U[1, max_q], seqlen_k = seqlen_q + U[0, max_extra_k] (int64 lists)."""
     g = torch.Generator().manual_seed(seed)

@@ -70,7 +70,7 @@ def _fwd(lib_b, **kw):
     B = lib_b
     p = B.FwdParams()
     p.struct_size = ctypes.sizeof(p)
-    p.version = 2
+    p.version = B.PARAMS_VERSION
     p.dtype = B.DTYPE_BF16
     p.B, p.H, p.Sq, p.Sk, p.D = 2, 3, 100, 90, 64
     p.q = p.k = p.v = p.o = p.lse = FAKE
@@ -89,7 +89,7 @@ def _call_fwd(B, p):
 
 
 @pytest.mark.parametrize("field,value", [
-    ("struct_size", 8), ("version", 3), ("version", 1), ("dtype", 2), ("D", 144), ("D", 0),
+    ("struct_size", 8), ("version", 4), ("version", 2), ("version", 1), ("dtype", 2), ("D", 144), ("D", 0),
     ("D", -3),
     ("B", -1), ("Sq", 1 << 30), ("sm_scale", float("nan")), ("sm_scale", float("inf")),
     ("varlen_bits", 1 << 19), ("varlen_bits", 1 << 31), ("varlen_bits", 0x20),
@@ -102,6 +102,7 @@ def _call_fwd(B, p):
     ("q", 0), ("o", 0), ("k", 0), ("q", FAKE + 8), ("o", FAKE + 2),
     ("q_stride", (3 * 128 * 64, 128 * 64, 60)),  # row stride of 120 bytes
     ("k_stride", (3 * 128 * 64, 0, 64)),         # zero head stride with H > 1
+    ("bias", FAKE + 8),                          # bias base not 16-byte aligned
 ])
 def test_forward_rejects_invalid_parameters(B, field, value):
     assert _call_fwd(B, _fwd(B, **{field: value})) == B.ERROR_INVALID_VALUE
@@ -122,12 +123,59 @@ def test_version_one_callers_are_accepted(B):
         == B.lib().attn_bwd_workspace_size(ctypes.byref(_bwd(B)))
 
 
-def test_header_version_one_sizes_match_the_binding(B):
+def test_version_two_callers_are_accepted(B):
+    # version 2 (no bias fields): validated without reading past its size
+    p = _fwd(B, B=0, version=2, struct_size=B.FWD_PARAMS_V2_SIZE, bias=FAKE + 2)
+    assert _call_fwd(B, p) == 0
+    q = _bwd(B, B=0, version=2, struct_size=B.BWD_PARAMS_V2_SIZE, dbias=FAKE + 2)
+    assert B.lib().attn_bwd(ctypes.byref(q), None) == 0
+    assert B.lib().attn_bwd_workspace_size(ctypes.byref(_bwd(B, version=2,
+                                                            struct_size=B.BWD_PARAMS_V2_SIZE))) \
+        == B.lib().attn_bwd_workspace_size(ctypes.byref(_bwd(B)))
+    # a version-2 number with the current size (or the reverse) is refused
+    assert _call_fwd(B, _fwd(B, B=0, version=2)) == B.ERROR_INVALID_VALUE
+    assert _call_fwd(B, _fwd(B, B=0, struct_size=B.FWD_PARAMS_V2_SIZE)) == B.ERROR_INVALID_VALUE
+
+
+def test_header_older_struct_sizes_match_the_binding(B):
     text = open(HEADER).read()
     assert "offsetof(attn_fwd_params, seqused_q)" in text
     assert "offsetof(attn_bwd_params, seqused_q)" in text
+    assert "offsetof(attn_fwd_params, bias)" in text
+    assert "offsetof(attn_bwd_params, bias)" in text
     assert B.FwdParams.seqused_q.offset == B.FWD_PARAMS_V1_SIZE
     assert B.BwdParams.seqused_q.offset == B.BWD_PARAMS_V1_SIZE
+    assert B.FwdParams.bias.offset == B.FWD_PARAMS_V2_SIZE
+    assert B.BwdParams.bias.offset == B.BWD_PARAMS_V2_SIZE
+
+
+BIAS_STRIDES = (3 * 100 * 96, 100 * 96, 96)   # [B=2, H=3, Sq=100, Sk=90] rows padded to 96
+
+
+@pytest.mark.parametrize("strides", [
+    (3 * 100 * 96, 100 * 96, 90),     # row stride of 180 bytes
+    (3 * 100 * 96, 100 * 96, 0),      # every query row on one row
+    (3 * 100 * 96, 100 * 96 + 4, 96), # head stride of odd 8-byte multiple
+    (-96, 100 * 96, 96),              # negative batch stride
+])
+def test_bias_strides_rejected(B, strides):
+    p = _fwd(B, bias=FAKE, bias_stride=strides)
+    assert _call_fwd(B, p) == B.ERROR_INVALID_VALUE
+    q = _bwd(B, workspace_bytes=1 << 30, bias=FAKE, bias_stride=strides)
+    assert B.lib().attn_bwd(ctypes.byref(q), None) == B.ERROR_INVALID_VALUE
+
+
+@pytest.mark.parametrize("strides", [(0, 100 * 96, 96), (3 * 100 * 96, 0, 96), (0, 0, 96)])
+def test_bias_broadcast_passes_validation_but_dbias_broadcast_does_not(B, strides):
+    # validation passes (the call then fails only for want of a device here)
+    p = _fwd(B, bias=FAKE, bias_stride=strides)
+    assert _call_fwd(B, p) != B.ERROR_INVALID_VALUE
+    q = _bwd(B, workspace_bytes=1 << 30, bias=FAKE, bias_stride=strides)
+    assert B.lib().attn_bwd(ctypes.byref(q), None) != B.ERROR_INVALID_VALUE
+    q = _bwd(B, workspace_bytes=1 << 30, dbias=FAKE, dbias_stride=strides)
+    assert B.lib().attn_bwd(ctypes.byref(q), None) == B.ERROR_INVALID_VALUE
+    q = _bwd(B, workspace_bytes=1 << 30, dbias=FAKE + 8, dbias_stride=BIAS_STRIDES)
+    assert B.lib().attn_bwd(ctypes.byref(q), None) == B.ERROR_INVALID_VALUE
 
 
 @pytest.mark.parametrize("mode_name", ["MODE_PACKED_USED", "MODE_PACKED_OFFSETS"])
@@ -165,7 +213,7 @@ def _bwd(lib_b, **kw):
     B = lib_b
     p = B.BwdParams()
     p.struct_size = ctypes.sizeof(p)
-    p.version = 2
+    p.version = B.PARAMS_VERSION
     p.dtype = B.DTYPE_FP16
     p.B, p.H, p.Sq, p.Sk, p.D = 2, 3, 100, 90, 128
     for n in ("q", "k", "v", "o", "dout", "lse", "dq", "dk", "dv", "workspace"):
