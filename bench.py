@@ -279,11 +279,14 @@ class Step:
         self.bias = self.dbias = None
         if bias:
             # [B, H, Sq, Sk] (largest lengths for packed inputs), drawn on the
-            # device: N(0, 1) from a seeded device generator
-            shape = (pr.B, w.H, pr.Sq, pr.Sk)
+            # device: N(0, 1) from a seeded device generator; rows are padded
+            # to a multiple of 8 elements (16-byte row strides)
+            pitch = (pr.Sk + 7) // 8 * 8
+            shape = (pr.B, w.H, pr.Sq, pitch)
             g = torch.Generator(device=dev).manual_seed(w.seed + 1)
-            self.bias = torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(dtype)
-            self.dbias = torch.empty_like(self.bias)
+            self.bias = torch.randn(shape, generator=g, device=dev,
+                                    dtype=torch.float32).to(dtype)[..., :pr.Sk]
+            self.dbias = torch.empty(shape, device=dev, dtype=dtype)[..., :pr.Sk]
             self.kw["bias"] = self.bias
         self.bp = B.bwd_params(self.do, self.q, self.k, self.v, self.o, self.lse, pr, self.dq,
                                self.dk, self.dv, bias=self.bias, dbias=self.dbias)

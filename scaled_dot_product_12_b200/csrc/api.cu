@@ -213,6 +213,29 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 4-D map over a [B, H, Sq, Sk] bias (the strides checked by
+// bias_strides_ok): dimensions (Sk, Sq, H, B), 64 x 128 boxes with 128-byte
+// swizzle, a head or batch dimension of stride 0 (broadcast) or extent 1 given
+// extent 1 (the kernel then uses coordinate 0: *h_bcast / *b_bcast).
+cudaError_t make_bias_map(CUtensorMap* map, const void* base, int Sq, int Sk, int H, int B,
+                          const int64_t* st, int32_t* h_bcast, int32_t* b_bcast) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const bool hb = H <= 1 || st[1] == 0, bb = B <= 1 || st[0] == 0;
+  cuuint64_t dims[4] = {(cuuint64_t)(Sk > 0 ? Sk : 1), (cuuint64_t)(Sq > 0 ? Sq : 1),
+                        (cuuint64_t)(hb ? 1 : H), (cuuint64_t)(bb ? 1 : B)};
+  cuuint64_t strides[3] = {dims[1] > 1 ? (cuuint64_t)(st[2] * 2) : 16,
+                           hb ? 16 : (cuuint64_t)(st[1] * 2), bb ? 16 : (cuuint64_t)(st[0] * 2)};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  *h_bcast = hb ? 1 : 0;
+  *b_bcast = bb ? 1 : 0;
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // 2-D fp32 map over the dQ accumulator [H*rows][D] (row pitch DA*4 bytes),
 // 32 x 32 boxes with 128-byte swizzle: the backward adds staged dQ tiles
 // through it.
@@ -349,6 +372,11 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
     set_dropout(a, p);
     a.bias = p->bias;
     for (int i = 0; i < 3; ++i) a.bias_stride[i] = p->bias_stride[i];
+    if (p->bias) {
+      e = make_bias_map(&a.tb, p->bias, p->Sq, p->Sk, p->H, p->B, p->bias_stride, &a.bias_h_bcast,
+                        &a.bias_b_bcast);
+      if (e != cudaSuccess) return e;
+    }
     return attn::launch_fwd(a, stream);
   });
 }

@@ -587,10 +587,15 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     // Bias and dbias columns of key j (null past the sequence, or when not
     // given): element (i, j) at col + i * stride.
     const uint16_t* bcol = nullptr;
+    const uint16_t* bwarp = nullptr;  // this warp's first key column (L2 prefetch)
     uint16_t* dbcol = nullptr;
     const int32_t sqb = min(sq, a.Sq);  // bias rows: never past the tensor's Sq
-    (void)sqb;
+    (void)sqb, (void)bwarp;
     if constexpr (BIAS) {
+      const int32_t j0 = n0 + quad * 32;
+      if (a.bias && j0 < min(sk, a.Sk))
+        bwarp = reinterpret_cast<const uint16_t*>(a.bias) + (int64_t)b * a.bias_stride[0] +
+                (int64_t)h * a.bias_stride[1] + j0;
       if (j < sk && j < a.Sk && a.bias)
         bcol = reinterpret_cast<const uint16_t*>(a.bias) + (int64_t)b * a.bias_stride[0] +
                (int64_t)h * a.bias_stride[1] + j;
@@ -698,6 +703,20 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       mbar_arrive_warp(x_ready);
     }
     float v_next = n_it > 1 ? row_val(1) : 0.f;  // this group's value for tile it + 1
+    // Bias: raw 16-bit values of key j for 16 queries from i0 (0 past the
+    // sequence), two sub-chunks in flight.
+    uint32_t braw[2][BIAS ? 16 : 1];
+    auto load_bias16 = [&](uint32_t (&dst)[BIAS ? 16 : 1], int32_t i0) {
+      if constexpr (BIAS) {
+        const uint16_t* p = bcol ? bcol + (int64_t)i0 * a.bias_stride[2] : nullptr;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          dst[k] = (p && i0 + k < sqb) ? (uint32_t)__ldg(p + (int64_t)k * a.bias_stride[2]) : 0u;
+      } else {
+        (void)dst, (void)i0;
+      }
+    };
+    load_bias16(braw[0], mb * 128 + qo);
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
       const int32_t m0 = (mb + it) * 128;
@@ -714,43 +733,68 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
       if constexpr (DROPOUT) stage_delta(it);
       if constexpr (BIAS) {
-        // the next tile's bias column into L2 (rows qo .. qo + 63 of it)
-        if (bcol && it + 1 < n_it) {
+        // the next tile's bias into L2: this warp's 32 key columns (64
+        // bytes of a row) for the group's 64 query rows, two rows per lane
+        if (bwarp && it + 1 < n_it) {
           const int32_t i1 = m0 + 128 + qo;
-          const int nr = min(64, sqb - i1);
-          const uint16_t* p = bcol + (int64_t)i1 * a.bias_stride[2];
-          for (int k = lane & 1; k < nr; k += 2)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (int64_t)k * a.bias_stride[2]));
+#pragma unroll
+          for (int k = lane; k < 64; k += 32)
+            if (i1 + k < sqb)
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(bwarp + (int64_t)(i1 + k) * a.bias_stride[2]));
         }
       }
+      if constexpr (BIAS) {
+        // Sub-chunks of 16 queries; each one's bias values are requested one
+        // sub-chunk ahead (the first of the next tile at the end of this
+        // one), so the loads overlap the exponentials.
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if constexpr (DROPOUT) keep[c] = keep_bits(it, c);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int sc = 2 * c + hh;
+            if (sc < 3)
+              load_bias16(braw[(sc + 1) & 1], m0 + qo + 16 * (sc + 1));
+            else if (it + 1 < n_it)
+              load_bias16(braw[0], m0 + 128 + qo);
+            uint32_t sr[16], half8[8];
+            tmem_ld16(tS + qo + 16 * sc, sr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int q0 = qo + 16 * sc + 2 * e, q1 = q0 + 1;
+              const float b0 = h16_to_f32<BF16>(braw[sc & 1][2 * e]) * 1.4426950408889634f;
+              const float b1 = h16_to_f32<BF16>(braw[sc & 1][2 * e + 1]) * 1.4426950408889634f;
+              float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, b0));
+              float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, b1));
+              if (!full) {
+                v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
+                v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
+              }
+              pk[16 * c + 8 * hh + e] = pack2<BF16>(v0, v1);
+              if constexpr (DROPOUT) {
+                const int kb = 16 * hh + 2 * e;  // bit of the 32-query chunk
+                v0 = (keep[c] >> kb) & 1u ? v0 : 0.f;
+                v1 = (keep[c] >> (kb + 1)) & 1u ? v1 : 0.f;
+                half8[e] = pack2<BF16>(v0, v1);
+              } else {
+                half8[e] = pk[16 * c + 8 * hh + e];
+              }
+            }
+            tmem_st8(tS + po + 16 * c + 8 * hh, half8);
+          }
+        }
+      } else {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         if constexpr (DROPOUT) keep[c] = keep_bits(it, c);
-        // bias(i, j) of the chunk's 32 queries, times log2(e); 0 past seqlen_q
-        float bl[BIAS ? 32 : 1];
-        if constexpr (BIAS) {
-          const int32_t i0 = m0 + qo + 32 * c;
-          const uint16_t* p = bcol ? bcol + (int64_t)i0 * a.bias_stride[2] : nullptr;
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            bl[k] = (p && i0 + k < sqb)
-                        ? h16_to_f32<BF16>(__ldg(p + (int64_t)k * a.bias_stride[2])) * 1.4426950408889634f
-                        : 0.f;
-        }
         uint32_t sr[32];
         tmem_ld32(tS + qo + 32 * c, sr);
         uint32_t chunk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int q0 = qo + 32 * c + 2 * e, q1 = q0 + 1;
-          float v0, v1;
-          if constexpr (BIAS) {
-            v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, bl[2 * e]));
-            v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, bl[2 * e + 1]));
-          } else {
-            v0 = ex2(__uint_as_float(sr[2 * e]) * sl2);
-            v1 = ex2(__uint_as_float(sr[2 * e + 1]) * sl2);
-          }
+          float v0 = ex2(__uint_as_float(sr[2 * e]) * sl2);
+          float v1 = ex2(__uint_as_float(sr[2 * e + 1]) * sl2);
           if (!full) {
             v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
             v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
@@ -765,6 +809,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           }
         }
         tmem_st16(tS + po + 16 * c, chunk);
+      }
       }
       if (half == 0) {
         // S^T(it) has been read: the operand can take tile it+1's terms.

@@ -342,6 +342,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       ATTN_W8(0), ATTN_W8(8)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               ATTN_W8(0)
+               : "memory");
+}
 #undef ATTN_W8
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -465,17 +470,6 @@ __device__ __forceinline__ void zero_row16(uint8_t* row, int ncols, int t, int n
     *reinterpret_cast<uint16_t*>(row + 2 * col) = 0;
 }
 
-// Eight 16-bit values at p (16-byte aligned) as four packed pairs, only the
-// first `ncols` of them read (the others, and all of them when ncols <= 0,
-// are 0).  Read-only data: the non-coherent path.
-__device__ __forceinline__ uint4 ld_row8(const uint16_t* p, int ncols) {
-  if (ncols >= 8) return __ldg(reinterpret_cast<const uint4*>(p));
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    if (e < ncols) w[e >> 1] |= (uint32_t)__ldg(p + e) << (16 * (e & 1));
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
 // A 16-bit value as fp32.
 template <bool BF16>
 __device__ __forceinline__ float h16_to_f32(uint32_t bits) {
@@ -485,14 +479,6 @@ __device__ __forceinline__ float h16_to_f32(uint32_t bits) {
     return __half2float(__ushort_as_half((unsigned short)bits));
   }
 }
-// L2 prefetch of the 128-byte lines that hold the first, the 65th and the
-// last of `ncols` (1..128) consecutive 16-bit values at p.
-__device__ __forceinline__ void prefetch_row_l2(const uint16_t* p, int ncols) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-  if (ncols > 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 64));
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (ncols - 1)));
-}
-
 // A compile-time flag passed to generic lambdas (for `if constexpr` code
 // paths instantiated per call site).
 template <bool V>

@@ -35,11 +35,12 @@
 
 namespace attn {
 
-template <int NQ, int DPAD>
+template <int NQ, int DPAD, bool BIAS = false>
 struct FwdCfg {
   static constexpr int kSoftmaxWarps = 4 * NQ;
   static constexpr int kLoadWarp = kSoftmaxWarps;
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kBiasWarp = kSoftmaxWarps + 2;  // bias tile producer (with a bias)
   // One more full warpgroup after the softmax groups (TMA warp, MMA warp and
   // two spare warps), so registers can be moved between warpgroups.
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
@@ -53,16 +54,22 @@ struct FwdCfg {
   static constexpr int kTileBytes = 128 * DPAD * 2;        // one 128-row tile of Q, K or V
   // Sets of Q tiles: two at head dims up to 64 (the next unit's Q loads while
   // the current unit runs), one at 128 (shared memory holds no second set).
+  // With a bias, one 128 x 128 bias tile per query tile takes the room of
+  // K / V stages.
   static constexpr int kQBufs = DPAD == 128 ? 1 : 2;
-  static constexpr int kKStages = DPAD == 128 ? 3 : 4;
-  static constexpr int kVStages = DPAD == 128 ? 2 : 4;
+  static constexpr int kKStages = BIAS ? 2 : (DPAD == 128 ? 3 : 4);
+  static constexpr int kVStages = BIAS ? (DPAD == 128 ? 1 : 2) : (DPAD == 128 ? 2 : 4);
+  static constexpr int kBiasTileBytes = BIAS ? 128 * 128 * 2 : 0;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBufs * NQ * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kOffB = kOffV + kVStages * kTileBytes;
+  static constexpr int kOffBar = kOffB + NQ * kBiasTileBytes;
   // barriers: q_full[QB][NQ] q_empty[QB] k_full[KS] k_empty[KS] v_full[VS]
   //           v_empty[VS] s_full[NQ] p_ready[NQ] o_done[NQ] mma_done
-  static constexpr int kNumBars = kQBufs * (NQ + 1) + 2 * kKStages + 2 * kVStages + 3 * NQ + 1;
+  //           b_full[NQ] b_empty[NQ]
+  static constexpr int kNumBars =
+      kQBufs * (NQ + 1) + 2 * kKStages + 2 * kVStages + 3 * NQ + 1 + 2 * NQ;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kTmemCols = (128 * NQ + DPAD * NQ) <= 256 ? 256 : 512;
@@ -93,7 +100,8 @@ __device__ __forceinline__ void fwd_issue_s(uint32_t d, uint32_t qd, uint32_t kd
 }
 
 // One work unit: query rows [m0, m0 + 128 nt) of sequence b, head h, as nt
-// query tiles (NQ, or 1 for the halves of a split unit).
+// query tiles (NQ; 1 for the halves of a split unit or where the sequence ends
+// within the first tile of its last block).
 struct FwdUnit {
   int32_t h, b, m0, nt, sq, sk, qrow0, krow0, bq, bk, nb, n_tiles;
   SeqWindow win;
@@ -171,6 +179,10 @@ __device__ __forceinline__ bool fwd_unit(const FwdArgs& a, int32_t n_mblocks, co
   }
   w.m0 = (n_mblocks - 1 - mrev) * 128 * NQ + 128 * half;
   if (w.m0 >= w.sq) return false;
+  // a unit takes only the query tiles that hold rows of the sequence (the
+  // last block of a sequence whose length is not a multiple of 128 NQ may
+  // need fewer)
+  w.nt = min(w.nt, (w.sq - w.m0 + 127) / 128);
   w.win = seq_window(a.wl, a.wr, a.bottom_right != 0, w.sq, w.sk);
   int32_t ne;
   fwd_tile_range(w.win, w.sq, w.sk, w.m0, 128 * w.nt, &w.nb, &ne);
@@ -179,9 +191,9 @@ __device__ __forceinline__ bool fwd_unit(const FwdArgs& a, int32_t n_mblocks, co
 }
 
 template <int NQ, int DPAD, bool BF16, bool DROPOUT, bool BIAS>
-__global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ FwdArgs args) {
-  using C = FwdCfg<NQ, DPAD>;
+  using C = FwdCfg<NQ, DPAD, BIAS>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
@@ -229,6 +241,9 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
   auto p_ready = [&](int t) { return bar0 + 8 * (bs + NQ + t); };
   auto o_done = [&](int t) { return bar0 + 8 * (bs + 2 * NQ + t); };
   const uint32_t mma_done = bar0 + 8 * (bs + 3 * NQ);
+  auto b_full = [&](int t) { return bar0 + 8 * (bs + 3 * NQ + 1 + t); };
+  auto b_empty = [&](int t) { return bar0 + 8 * (bs + 4 * NQ + 1 + t); };
+  const uint32_t sB = sbase + C::kOffB;  // bias tile of query tile t at sB + t * 32 KiB
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -251,6 +266,10 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       mbar_init(v_empty(s), 1);
     }
     mbar_init(mma_done, 1);
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(b_full(t), 1);
+      mbar_init(b_empty(t), 4);  // one arrival per softmax warp of the tile
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -456,6 +475,41 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       tc_commit(mma_done);
       mbar_drain(mma_done, 0, args.status);
     }
+  } else if (BIAS && warp == C::kBiasWarp) {
+    // ===================== bias tile producer =====================
+    // The bias tile (query tile t, key tile) of every unit, in the order the
+    // softmax groups take them: one buffer per query tile, refilled as soon
+    // as the group has added the previous tile to its scores.  A thread of
+    // its own, so no K / V wait delays a bias load.
+    if (lane == 0) {
+      prefetch_tmap(&args.tb);
+      int64_t nbt[NQ] = {};  // bias tiles issued per query tile
+      bool stop = false;
+      for (int64_t u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
+        FwdUnit w;
+        if (!fwd_unit<NQ>(args, n_mblocks, units, u, w) || w.n_tiles <= 0) continue;
+        const int cb = args.bias_b_bcast ? 0 : w.b, ch = args.bias_h_bcast ? 0 : w.h;
+        for (int it = 0; it < w.n_tiles && !stop; ++it) {
+          const int n0 = (w.nb + it) * 128;
+          for (int t = 0; t < w.nt; ++t) {
+            if (nbt[t] > 0 && !mbar_wait(b_empty(t), (uint32_t)((nbt[t] - 1) & 1), abort_flag,
+                                         args.status, kSiteLoad)) {
+              stop = true;
+              break;
+            }
+            mbar_expect_tx(b_full(t), C::kBiasTileBytes);
+            for (int blk = 0; blk < 2; ++blk)
+              tma_load_4d(sB + t * C::kBiasTileBytes + blk * 16384, &args.tb, b_full(t),
+                          n0 + 64 * blk, w.m0 + 128 * t, ch, cb);
+            ++nbt[t];
+          }
+        }
+      }
+      if (*abort_flag) {
+        for (int t = 0; t < NQ; ++t)
+          if (nbt[t] > 0) mbar_drain(b_full(t), (uint32_t)((nbt[t] - 1) & 1), args.status);
+      }
+    }
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kHighRegs));
@@ -486,56 +540,47 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
       const int32_t lo = row_lo(w.win, i), hi = row_hi(w.win, i, w.sk);
       const uint32_t bh = (uint32_t)(w.b * args.H + w.h);  // dropout counter word
       (void)bh;
-      // Bias row of query i (null past the sequence, or past the bias
-      // tensor's Sq rows for an over-long sequence: those rows read 0).
-      const uint16_t* brow = nullptr;
-      if constexpr (BIAS) {
-        if (valid && i < args.Sq)
-          brow = reinterpret_cast<const uint16_t*>(args.bias) + (int64_t)w.b * args.bias_stride[0] +
-                 (int64_t)w.h * args.bias_stride[1] + (int64_t)i * args.bias_stride[2];
-      }
       // With a bias the logits are formed in the log2 domain below
       // (c S log2(e) + B log2(e)), and the shift works at unit scale.
       const float sl2e = BIAS ? 1.f : sl2;
+      // Row r of this tile's staged bias (128-byte swizzled 64-column blocks).
+      const uint32_t brow_s = sB + t * C::kBiasTileBytes + r * 128;
+      (void)brow_s;
       float m_used = -INFINITY, l = 0.f;
       for (int it = 0; it < w.n_tiles; ++it) {
         const int64_t gi = g + it;
         const int32_t n0 = (w.nb + it) * 128;
-        // The tile's bias (columns n0 .. n0 + 127, those past seqlen_k read
-        // as 0) is requested before the wait for S, and the next tile's
-        // lines are prefetched into L2.
-        uint4 bq[BIAS ? 16 : 1];
-        if constexpr (BIAS) {
-          const int32_t left = brow ? min(w.sk, args.Sk) - n0 : 0;
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            bq[q] = left > 8 * q ? ld_row8(brow + n0 + 8 * q, left - 8 * q) : make_uint4(0, 0, 0, 0);
-          if (brow && it + 1 < w.n_tiles && left > 128)
-            prefetch_row_l2(brow + n0 + 128, min(left - 128, 128));
-        }
         ok = mbar_wait(s_full(t), (uint32_t)(gi & 1), abort_flag, args.status, kSiteSoftmax);
+        if (BIAS && ok)
+          ok = mbar_wait(b_full(t), (uint32_t)(gi & 1), abort_flag, args.status, kSiteSoftmax);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
         float s[128];
         if constexpr (BIAS) {
-          // Four TMEM loads of 32 columns, each folded with its bias columns
-          // at once, so the raw scores and the bias are never all live.
+          // Four TMEM loads of 32 columns, each folded with its 32 bias
+          // columns (rows past the tensor read TMA's zero fill; rows past the
+          // sequence are not stored).
 #pragma unroll
           for (int part = 0; part < 4; ++part) {
             uint32_t raw[32];
             tmem_ld32(tS + 32 * part, raw);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 v = bq[4 * part + q];
-              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+              const int ch = 4 * part + q;  // 16-byte chunk of the row, 0..15
+              uint32_t wv[4];
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(wv[0]), "=r"(wv[1]), "=r"(wv[2]), "=r"(wv[3])
+                           : "r"(brow_s + (ch >> 3) * 16384 + (((ch & 7) ^ (r & 7)) << 4)));
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const int c = 32 * part + 8 * q + e;
+                const int c = 8 * ch + e;
                 const float bias = h16_to_f32<BF16>((wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
                 s[c] = fmaf(__uint_as_float(raw[8 * q + e]), sl2, bias * 1.4426950408889634f);
               }
             }
           }
+          // the bias tile has been read: its buffer can take the next one
+          mbar_arrive_warp(b_empty(t));
         } else {
           // The whole score row in one TMEM load.
           uint32_t raw[128];
@@ -678,7 +723,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD>::kThreads, 1)
 
 template <int NQ, int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 static cudaError_t launch(const FwdArgs& args, int64_t n_units, cudaStream_t stream) {
-  using C = FwdCfg<NQ, DPAD>;
+  using C = FwdCfg<NQ, DPAD, BIAS>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   static_assert(NQ * 128 * C::kHighRegs + 128 * C::kLowRegs <= C::kThreads * C::kLaunchRegs,
                 "register split exceeds the launch budget");

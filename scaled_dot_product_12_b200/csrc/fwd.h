@@ -43,9 +43,13 @@ struct FwdArgs {
   uint32_t keep_below, seed_lo, seed_hi, philox_offset;
   float drop_scale;
   // Additive bias: element (b, h, i, j) of sequence b at bias + b*s[0] +
-  // h*s[1] + i*s[2] + j (16-bit, the dtype of Q), or null.
+  // h*s[1] + i*s[2] + j (16-bit, the dtype of Q), or null.  The forward
+  // stages it through `tb`, a 4-D map (Sk, Sq, heads, batches) whose head /
+  // batch extent is 1 where that stride is 0 (the *_bcast flags: coordinate 0).
   const void* bias;
   int64_t bias_stride[3];
+  CUtensorMap tb;
+  int32_t bias_b_bcast, bias_h_bcast;
 };
 
 struct BwdArgs {
