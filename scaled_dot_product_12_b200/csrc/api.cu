@@ -528,6 +528,11 @@ int attn_bwd(const attn_bwd_params* params, void* stream_ptr) {
       a.bias_stride[i] = p->bias_stride[i];
       a.dbias_stride[i] = p->dbias_stride[i];
     }
+    if (p->bias) {
+      e = make_bias_map(&a.tb, p->bias, p->Sq, p->Sk, p->H, p->B, p->bias_stride, &a.bias_h_bcast,
+                        &a.bias_b_bcast);
+      if (e != cudaSuccess) return e;
+    }
     a.main_events[0] = static_cast<cudaEvent_t>(p->main_kernel_events[0]);
     a.main_events[1] = static_cast<cudaEvent_t>(p->main_kernel_events[1]);
     return attn::launch_bwd(a, stream);

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(256) attn_dq_convert_seq_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // 2. main backward
 // ---------------------------------------------------------------------------
-template <int DPAD>
+template <int DPAD, bool BIAS = false>
 struct BwdCfg {
   // Warps 0-7: two P/dS groups (query columns 0-63 and 64-127 of every key
   // row); 8-11: dQ drain; 12: TMA; 13: MMA; 14-15 idle.  16 warps, four per
@@ -207,11 +207,17 @@ struct BwdCfg {
   // dP^T tile, on the query side.
   static constexpr int kXBytes = 128 * 16 * 2;
   static constexpr int kOffX = kOffDQ + kDqStageBytes;
-  static constexpr int kOffBar = kOffX + 3 * kXBytes;
+  // With a bias at head dim 64, the bias tile of the current query tile
+  // (128 queries x 128 keys, 16-bit, two 128-byte swizzled 64-key blocks) is
+  // staged by TMA; at 128 there is no room and the P / dS warps load it.
+  static constexpr bool kStageBias = BIAS && DPAD == 64;
+  static constexpr int kBiasTileBytes = kStageBias ? 128 * 128 * 2 : 0;
+  static constexpr int kOffBias = kOffX + 3 * kXBytes;
+  static constexpr int kOffBar = kOffBias + kBiasTileBytes;
   // kv_full, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
   // dp_full, p_ready, ds_ready, dq_mma, dq_free, acc_done, x_ready,
-  // delta_ready[2]
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 10;
+  // delta_ready[2], b_full, b_empty
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDOStages + 12;
   // With dropout, delta is not folded into dP^T: each P/dS group stages the
   // delta values of its 64 query columns, two tiles deep.
   static constexpr int kOffDelta = kOffBar + 8 * kNumBars;
@@ -265,7 +271,7 @@ __device__ __forceinline__ void bwd_issue_mn(uint32_t d, uint32_t a_lo, uint32_t
 
 template <int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
-  using C = BwdCfg<DPAD>;
+  using C = BwdCfg<DPAD, BIAS>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
@@ -359,6 +365,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
                  dq_mma = s_full + 32, dq_free = s_full + 40, acc_done = s_full + 48,
                  x_ready = s_full + 56;
   auto delta_ready = [&](int g) { return s_full + 64 + 8 * g; };
+  const uint32_t b_full = s_full + 80, b_empty = s_full + 88;  // staged bias tile
+  const uint32_t sBias = sbase + C::kOffBias;
+  (void)b_full, (void)b_empty, (void)sBias;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -382,6 +391,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(x_ready, 8);
     mbar_init(delta_ready(0), 4);  // one per warp of the group
     mbar_init(delta_ready(1), 4);
+    mbar_init(b_full, 1);
+    mbar_init(b_empty, 8);  // one per P / dS warp
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -562,10 +573,31 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         issue_all(Flag<false>{});
     }
   } else if (BIAS) {
-    // Warps 14-15: dbias of the query rows outside the visited tiles.
-    const int t = (warp - 14) * 32 + lane;
-    zero_dbias_rows(0, min(mb * 128, sq), t, 64);
-    zero_dbias_rows(min(me * 128, sq), sq, t, 64);
+    if (C::kStageBias && warp == 14) {
+      // ===================== bias tile producer (head dim 64) =====================
+      // The bias tile of each visited query tile (query rows x this CTA's
+      // keys) into shared memory, refilled as soon as the P / dS warps have
+      // read the previous one.
+      if (lane == 0 && a.bias) {
+        prefetch_tmap(&a.tb);
+        const int cb = a.bias_b_bcast ? 0 : b, ch = a.bias_h_bcast ? 0 : h;
+        int it = 0;
+        for (; it < n_it; ++it) {
+          if (it > 0 && !mbar_wait(b_empty, (uint32_t)((it - 1) & 1), abort_flag, a.status, kSiteLoad))
+            break;
+          mbar_expect_tx(b_full, C::kBiasTileBytes);
+          for (int blk = 0; blk < 2; ++blk)
+            tma_load_4d(sBias + blk * 16384, &a.tb, b_full, n0 + 64 * blk, (mb + it) * 128, ch, cb);
+        }
+        if (*abort_flag && it > 0) mbar_drain(b_full, (uint32_t)((it - 1) & 1), a.status);
+      }
+    } else {
+      // dbias of the query rows outside the visited tiles
+      const int t = C::kStageBias ? lane : (warp - 14) * 32 + lane;
+      const int nt = C::kStageBias ? 32 : 64;
+      zero_dbias_rows(0, min(mb * 128, sq), t, nt);
+      zero_dbias_rows(min(me * 128, sq), sq, t, nt);
+    }
   }
   } else if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kPdsRegs));
@@ -707,7 +739,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     // sequence), two sub-chunks in flight.
     uint32_t braw[2][BIAS ? 16 : 1];
     auto load_bias16 = [&](uint32_t (&dst)[BIAS ? 16 : 1], int32_t i0) {
-      if constexpr (BIAS) {
+      if constexpr (BIAS && !C::kStageBias) {
         const uint16_t* p = bcol ? bcol + (int64_t)i0 * a.bias_stride[2] : nullptr;
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -723,7 +755,10 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       const bool full = tile_is_full(win, sq, sk, m0, n0);
       const int32_t ca = qa - m0, cz = qz - m0;  // allowed columns [ca, cz]
       // ---- phase 1: P^T = exp2(c * (S^T - LSE*log2(e)/c)), masked ----
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax));
+      ok = mbar_wait(s_full, it & 1, abort_flag, a.status, kSiteSoftmax);
+      if (C::kStageBias && ok && a.bias)
+        ok = mbar_wait(b_full, it & 1, abort_flag, a.status, kSiteSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       // P is kept as the rounded 16-bit pairs the dV product uses (with
@@ -732,7 +767,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       uint32_t pk[32];
       uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
       if constexpr (DROPOUT) stage_delta(it);
-      if constexpr (BIAS) {
+      if constexpr (BIAS && !C::kStageBias) {
         // the next tile's bias into L2: this warp's 32 key columns (64
         // bytes of a row) for the group's 64 query rows, two rows per lane
         if (bwarp && it + 1 < n_it) {
@@ -743,7 +778,52 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
               asm volatile("prefetch.global.L2 [%0];" ::"l"(bwarp + (int64_t)(i1 + k) * a.bias_stride[2]));
         }
       }
-      if constexpr (BIAS) {
+      if constexpr (C::kStageBias) {
+        // Staged bias tile: (query q of the tile, key r) at 64-key block
+        // r / 64, row q, 16-byte chunk ((r % 64) / 8) xor (q % 8), 2 bytes r % 8.
+        const uint32_t bcol_s = sBias + (r >> 6) * 16384 + (r & 7) * 2;
+        const uint32_t bchunk = (uint32_t)((r & 63) >> 3);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if constexpr (DROPOUT) keep[c] = keep_bits(it, c);
+          uint32_t sr[32];
+          tmem_ld32(tS + qo + 32 * c, sr);
+          uint32_t chunk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int q0 = qo + 32 * c + 2 * e, q1 = q0 + 1;
+            float b0 = 0.f, b1 = 0.f;
+            if (a.bias) {
+              uint16_t h0, h1;
+              asm volatile("ld.shared.u16 %0, [%1];"
+                           : "=h"(h0)
+                           : "r"(bcol_s + q0 * 128 + ((bchunk ^ (q0 & 7)) << 4)));
+              asm volatile("ld.shared.u16 %0, [%1];"
+                           : "=h"(h1)
+                           : "r"(bcol_s + q1 * 128 + ((bchunk ^ (q1 & 7)) << 4)));
+              b0 = h16_to_f32<BF16>(h0) * 1.4426950408889634f;
+              b1 = h16_to_f32<BF16>(h1) * 1.4426950408889634f;
+            }
+            float v0 = ex2(fmaf(__uint_as_float(sr[2 * e]), sl2, b0));
+            float v1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, b1));
+            if (!full) {
+              v0 = (q0 < ca || q0 > cz) ? 0.f : v0;
+              v1 = (q1 < ca || q1 > cz) ? 0.f : v1;
+            }
+            pk[16 * c + e] = pack2<BF16>(v0, v1);
+            if constexpr (DROPOUT) {
+              v0 = (keep[c] >> (2 * e)) & 1u ? v0 : 0.f;
+              v1 = (keep[c] >> (2 * e + 1)) & 1u ? v1 : 0.f;
+              chunk[e] = pack2<BF16>(v0, v1);
+            } else {
+              chunk[e] = pk[16 * c + e];
+            }
+          }
+          tmem_st16(tS + po + 16 * c, chunk);
+        }
+        // the bias tile has been read: the producer can load the next one
+        if (a.bias) mbar_arrive_warp(b_empty);
+      } else if constexpr (BIAS) {
         // Sub-chunks of 16 queries; each one's bias values are requested one
         // sub-chunk ahead (the first of the next tile at the end of this
         // one), so the loads overlap the exponentials.
@@ -1030,7 +1110,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
 
 template <int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 static cudaError_t launch_main(const BwdArgs& a, cudaStream_t stream) {
-  using C = BwdCfg<DPAD>;
+  using C = BwdCfg<DPAD, BIAS>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   // One warp of each warpgroup per sub-partition: P/dS, P/dS, drain, TMA/MMA.
   static_assert(2 * C::kPdsRegs + C::kDrainRegs + C::kProducerRegs <= 4 * C::kLaunchRegs,

@@ -92,6 +92,8 @@ struct BwdArgs {
   const void* bias;
   void* dbias;
   int64_t bias_stride[3], dbias_stride[3];
+  CUtensorMap tb;  // as in FwdArgs (head dim 64 stages the bias tiles)
+  int32_t bias_b_bcast, bias_h_bcast;
 };
 
 cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream);

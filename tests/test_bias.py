@@ -113,11 +113,12 @@ def test_broadcast_bias(shape):
     assert_dbias(f64(dbias), edb, w)
 
 
-def test_dbias_without_bias_is_the_gradient_at_zero_bias():
+@pytest.mark.parametrize("D", [128, 64])
+def test_dbias_without_bias_is_the_gradient_at_zero_bias(D):
     B = binding()
-    Bn, H, Sq, Sk, D = 1, 2, 257, 300, 128
+    Bn, H, Sq, Sk = 1, 2, 257, 300
     dtype = torch.float16
-    q, k, v, do = synth.qkv_do((Bn, H, Sq, D), (Bn, H, Sk, D), seed_of("dbias0"), dtype)
+    q, k, v, do = synth.qkv_do((Bn, H, Sq, D), (Bn, H, Sk, D), seed_of("dbias0", D), dtype)
     w = (-10, 90, True)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     o, lse = B.forward(qd, kd, vd, sm_scale=0.1, window=w[:2], bottom_right=w[2])
@@ -157,15 +158,17 @@ def test_large_position_bias_moves_the_row_maximum():
     assert_dbias(f64(dbias), edb, (INF, INF, False))
 
 
+@pytest.mark.parametrize("D", [80, 64])
 @pytest.mark.parametrize("w", [(INF, INF, False), (CBR, 0, True), (-32, 64, True)], ids=str)
-def test_packed_bias(w):
+def test_packed_bias(w, D):
     # bias [B, H, max_q, max_k], (i, j) within each sequence; NaN past every
-    # sequence's lengths
+    # sequence's lengths (head dim 64 stages the bias tiles in shared memory,
+    # 80 loads them per thread)
     B = binding()
     sq, sk = [1, 130, 257, 64], [5, 300, 128, 64]
-    H, D, dtype = 2, 80, torch.bfloat16
+    H, dtype = 2, torch.bfloat16
     tq, tk = sum(sq), sum(sk)
-    q, k, v, do = synth.qkv_do((tq, H, D), (tk, H, D), seed_of("pbias", w), dtype)
+    q, k, v, do = synth.qkv_do((tq, H, D), (tk, H, D), seed_of("pbias", w, D), dtype)
     Mq, Mk = max(sq), max(sk)
     full = synth.bias((len(sq), H, Mq, Mk), seed_of("pbias-b", w), dtype, std=2.0)
     for s in range(len(sq)):
