@@ -34,7 +34,9 @@
 namespace attn {
 
 // ---------------------------------------------------------------------------
-// 1. preprocess: 16 threads per (head, row), 8 elements each.
+// 1. preprocess: TPR threads per (head, row) -- 8 when the head dims are at
+// most 64, else 16 -- each one 16-byte chunk of O and dO and 32 bytes of the
+// accumulator.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int64_t row_offset(const int64_t* st, int64_t row, int h, int Sq,
                                               bool packed) {
@@ -43,13 +45,14 @@ __device__ __forceinline__ int64_t row_offset(const int64_t* st, int64_t row, in
   return b * st[0] + (int64_t)h * st[1] + s * st[2];
 }
 
-template <bool BF16>
+template <bool BF16, int TPR>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant__ BwdArgs a) {
+  constexpr int kGroups = 256 / TPR;  // (head, row) groups per block and pass
   const int64_t n_groups = (int64_t)a.H * a.rows;
-  const int sub = threadIdx.x & 15;
+  const int sub = threadIdx.x & (TPR - 1);
   const int chunks = (a.Dv + 7) / 8;  // of O and dO, 8 columns each; the last may be partial
-  for (int64_t g = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4); g < n_groups;
-       g += (int64_t)gridDim.x * 16) {
+  for (int64_t g = (int64_t)blockIdx.x * kGroups + threadIdx.x / TPR; g < n_groups;
+       g += (int64_t)gridDim.x * kGroups) {
     const int h = (int)(g / a.rows);
     const int64_t row = g % a.rows;
     float acc = 0.f;
@@ -88,7 +91,7 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __grid_constant
       if (a.order && sub == 0) reinterpret_cast<int4*>(a.order)[g] = make_int4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int m = 8; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    for (int m = TPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
     if (sub == 0) a.delta[g] = acc;
   }
 }
@@ -1127,9 +1130,14 @@ template <bool BF16>
 static cudaError_t launch_all(const BwdArgs& a, cudaStream_t stream, int sms) {
   const int64_t groups = (int64_t)a.H * a.rows;
   if (groups > 0) {
-    const int64_t want = (groups + 15) / 16;
+    const bool narrow = a.Dv <= 64 && a.DA <= 64;  // 8 threads cover a row
+    const int per_block = narrow ? 32 : 16;
+    const int64_t want = (groups + per_block - 1) / per_block;
     const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-    attn_bwd_pre_kernel<BF16><<<grid, 256, 0, stream>>>(a);
+    if (narrow)
+      attn_bwd_pre_kernel<BF16, 8><<<grid, 256, 0, stream>>>(a);
+    else
+      attn_bwd_pre_kernel<BF16, 16><<<grid, 256, 0, stream>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
