@@ -35,7 +35,7 @@
 
 namespace attn {
 
-template <int NQ, int DPAD, bool BIAS = false>
+template <int NQ, int DPAD, bool BIAS = false, bool DROPOUT = false>
 struct FwdCfg {
   static constexpr int kSoftmaxWarps = 4 * NQ;
   static constexpr int kLoadWarp = kSoftmaxWarps;
@@ -46,9 +46,13 @@ struct FwdCfg {
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
   // Register split (setmaxnreg): the launch gives every thread kLaunchRegs;
   // the producer/MMA group drops to kLowRegs, the softmax groups rise to
-  // kHighRegs.  NQ*128*kHighRegs + 128*kLowRegs == kThreads*kLaunchRegs.
+  // kHighRegs.  NQ*128*kHighRegs + 128*kLowRegs <= kThreads*kLaunchRegs.  The
+  // low shares are the smallest the producer / MMA code compiles into without
+  // spilling, so the softmax (one 128-column score row per thread) gets the
+  // most: 192 at head dim 128, 200 at 64 (with dropout at 128 its Philox
+  // state needs the 136 / 184 split).
   static constexpr int kLaunchRegs = 168;  // 65536 / (4 sub-partitions x 3 warps x 32) rounded to 8
-  static constexpr int kLowRegs = 136;
+  static constexpr int kLowRegs = DPAD == 128 ? (DROPOUT ? 136 : 112) : 104;
   static constexpr int kHighRegs = (kThreads * kLaunchRegs - 128 * kLowRegs) / (128 * NQ) / 8 * 8;
   static constexpr int kBlocks = DPAD / 64;                // 128-byte swizzle blocks per row
   static constexpr int kTileBytes = 128 * DPAD * 2;        // one 128-row tile of Q, K or V
@@ -191,9 +195,9 @@ __device__ __forceinline__ bool fwd_unit(const FwdArgs& a, int32_t n_mblocks, co
 }
 
 template <int NQ, int DPAD, bool BF16, bool DROPOUT, bool BIAS>
-__global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS>::kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ FwdArgs args) {
-  using C = FwdCfg<NQ, DPAD, BIAS>;
+  using C = FwdCfg<NQ, DPAD, BIAS, DROPOUT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
@@ -723,7 +727,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS>::kThreads, 1)
 
 template <int NQ, int DPAD, bool BF16, bool DROPOUT, bool BIAS>
 static cudaError_t launch(const FwdArgs& args, int64_t n_units, cudaStream_t stream) {
-  using C = FwdCfg<NQ, DPAD, BIAS>;
+  using C = FwdCfg<NQ, DPAD, BIAS, DROPOUT>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   static_assert(NQ * 128 * C::kHighRegs + 128 * C::kLowRegs <= C::kThreads * C::kLaunchRegs,
                 "register split exceeds the launch budget");
