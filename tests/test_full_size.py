@@ -105,3 +105,46 @@ def test_packed_workload_count_probe(case):
         assert np.array_equal(np.isneginf(rows), np.broadcast_to(empty[:, None], rows.shape))
         got = np.rint(np.exp(rows[~empty]))
         assert np.array_equal(got, np.broadcast_to(cnt[~empty, None], got.shape).astype(float))
+
+
+@pytest.mark.parametrize("name,shared", [("bert_large", False), ("gpt2", False),
+                                         ("ltx_6630", True)])
+def test_dense_workload_with_bias_sampled_heads(name, shared):
+    """The additive bias and its gradient at full size: a bias per (batch,
+    head) for the D = 64 shapes (staged by TMA in both kernels), one bias
+    shared by every batch and head at LTX 6630 (D = 128: staged in the
+    forward, loaded per thread in the backward)."""
+    B = binding()
+    w = synth.WORKLOADS[name]
+    dtype = synth.DTYPES[w.dtype]
+    dev = torch.device("cuda")
+    q, k, v, do = synth.qkv_do((w.B, w.H, w.Sq, w.D), (w.B, w.H, w.Sk, w.D), w.seed, dtype)
+    pitch = (w.Sk + 7) // 8 * 8  # 16-byte rows
+    shape = (1, 1) if shared else (w.B, w.H)
+    host_bias = synth.bias(shape + (w.Sq, w.Sk), w.seed + 101, dtype, std=1.0)
+    bias_buf = torch.zeros(shape + (w.Sq, pitch), dtype=dtype, device=dev)
+    bias_buf[..., :w.Sk] = host_bias.to(dev)
+    bias = bias_buf[..., :w.Sk].expand(w.B, w.H, w.Sq, w.Sk)
+    dbias = torch.empty((w.B, w.H, w.Sq, pitch), dtype=dtype, device=dev)[..., :w.Sk]
+    scale = w.D ** -0.5
+    win = (w.window_left, w.window_right)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    kw = dict(sm_scale=scale, window=win, bottom_right=w.bottom_right, bias=bias)
+    o, lse = B.forward(qd, kd, vd, **kw)
+    dq, dk, dv, _ = B.backward(dod, qd, kd, vd, o, lse, dbias=dbias, **kw)
+    torch.cuda.synchronize()
+    assert B.device_status(dev) == 0
+    for b, h in _sample_heads(w, 1, w.seed + 7):
+        bb = f64(host_bias[0, 0] if shared else host_bias[b, h])
+        eo, el = ref.forward(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), scale, *win, w.bottom_right,
+                             bias=bb)
+        eg = ref.backward(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), f64(do[b, h]), scale, *win,
+                          w.bottom_right, bias=bb)
+        what = f"{name} bias head {(b, h)}"
+        assert_o_lse(o[b, h].float().cpu().numpy(), lse[b, h].cpu().numpy(), eo, el, dtype, what=what)
+        assert_grads([t[b, h].float().cpu().numpy() for t in (dq, dk, dv)], eg[:3], what=what)
+        got_db = dbias[b, h].float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(got_db).all()
+        assert_grads([got_db], [eg[3]], what=what + " dbias")
+        allowed = ref.allowed(w.Sq, w.Sk, *win, w.bottom_right)
+        assert (got_db[~allowed] == 0).all()
