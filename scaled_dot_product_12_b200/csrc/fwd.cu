@@ -71,13 +71,19 @@ struct FwdCfg {
   static constexpr int kOffBar = kOffB + NQ * kBiasTileBytes;
   // barriers: q_full[QB][NQ] q_empty[QB] k_full[KS] k_empty[KS] v_full[VS]
   //           v_empty[VS] s_full[NQ] p_ready[NQ] o_done[NQ] mma_done
-  //           b_full[NQ] b_empty[NQ]
+  //           b_full[NQ] b_empty[NQ] s_free[NQ]
   static constexpr int kNumBars =
-      kQBufs * (NQ + 1) + 2 * kKStages + 2 * kVStages + 3 * NQ + 1 + 2 * NQ;
+      kQBufs * (NQ + 1) + 2 * kKStages + 2 * kVStages + 3 * NQ + 1 + 3 * NQ;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16;
-  static constexpr int kTmemCols = (128 * NQ + DPAD * NQ) <= 256 ? 256 : 512;
-  static constexpr int kColO = 128 * NQ;
+  // TMEM: S of tile t at [128 t, 128 t + 128).  At head dims up to 64, P of
+  // tile t has columns of its own, [256 + 64 t, +64) as 16-bit pairs, so the
+  // next S product can overwrite S as soon as the softmax has read it (it runs
+  // while the softmax computes P); at 128 there is no room and P overwrites S.
+  static constexpr bool kSplitP = DPAD == 64 && NQ == 2;
+  static constexpr int kColP = kSplitP ? 128 * NQ : 0;
+  static constexpr int kColO = kSplitP ? 128 * NQ + 64 * NQ : 128 * NQ;
+  static constexpr int kTmemCols = (kColO + DPAD * NQ) <= 256 ? 256 : 512;
 };
 
 // O (+)= P V for one query tile: P from TMEM (8 columns per K step of 16
@@ -247,6 +253,9 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
   const uint32_t mma_done = bar0 + 8 * (bs + 3 * NQ);
   auto b_full = [&](int t) { return bar0 + 8 * (bs + 3 * NQ + 1 + t); };
   auto b_empty = [&](int t) { return bar0 + 8 * (bs + 4 * NQ + 1 + t); };
+  // split P: the softmax group of tile t has read S(t), which the next S
+  // product may overwrite
+  auto s_free = [&](int t) { return bar0 + 8 * (bs + 5 * NQ + 1 + t); };
   const uint32_t sB = sbase + C::kOffB;  // bias tile of query tile t at sB + t * 32 KiB
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -273,6 +282,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
     for (int t = 0; t < NQ; ++t) {
       mbar_init(b_full(t), 1);
       mbar_init(b_empty(t), 4);  // one arrival per softmax warp of the tile
+      mbar_init(s_free(t), 4);   // the same
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -405,7 +415,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
           };
           // O_t (+)= P_t V, then O_t's completion on o_done(t).
           auto issue_pv = [&](int t, int vs, bool accumulate) {
-            fwd_issue_pv(tmem + C::kColO + DPAD * t, tmem + 128 * t,
+            fwd_issue_pv(tmem + C::kColO + DPAD * t, tmem + (C::kSplitP ? C::kColP + 64 * t : 128 * t),
                          dV + (uint32_t)vs * kTile16, kHiV, idesc_o, accumulate);
             tc_commit(o_done(t));
           };
@@ -419,6 +429,52 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
             ok = mbar_wait(q_full(qb, t), (uint32_t)(qw[qb][t] & 1), abort_flag, args.status,
                            kSiteMma);
             ++qw[qb][t];
+          }
+          if constexpr (C::kSplitP) {
+            // S(t, it + 1) goes out as soon as the softmax has read S(t, it),
+            // before P V of tile it: the products of the next key tile run
+            // while the softmax computes P.
+            auto issue_s_tile = [&](int it) -> bool {  // S of key tile it, both query tiles
+              const int64_t gi = g + it;
+              const int ks = (int)(gi % C::kKStages);
+              if (!mbar_wait(k_full(ks), (uint32_t)((gi / C::kKStages) & 1), abort_flag,
+                             args.status, kSiteMma))
+                return false;
+              for (int t = 0; t < w.nt; ++t) {
+                const int64_t prev = gt[t] + it - 1;  // the S(t) the softmax must have read
+                if (prev >= 0 && !mbar_wait(s_free(t), (uint32_t)(prev & 1), abort_flag,
+                                            args.status, kSiteMma))
+                  return false;
+                tc_fence_after();
+                issue_s(t, ks);
+              }
+              tc_commit(k_empty(ks));
+              if (it == w.n_tiles - 1) tc_commit(q_empty(qb));
+              return true;
+            };
+            ok = issue_s_tile(0);
+            for (int it = 0; it < w.n_tiles && ok; ++it) {
+              if (it + 1 < w.n_tiles && !(ok = issue_s_tile(it + 1))) break;
+              const int64_t gi = g + it;
+              const int vs = (int)(gi % C::kVStages);
+              for (int t = 0; t < w.nt && ok; ++t) {
+                if (!(ok = mbar_wait(p_ready(t), (uint32_t)((gt[t] + it) & 1), abort_flag,
+                                     args.status, kSiteMma)))
+                  break;
+                if (t == 0) {
+                  if (!(ok = mbar_wait(v_full(vs), (uint32_t)((gi / C::kVStages) & 1), abort_flag,
+                                       args.status, kSiteMma)))
+                    break;
+                  clear_v_padding(it, vs);
+                }
+                tc_fence_after();
+                issue_pv(t, vs, it > 0);
+                if (t == w.nt - 1) tc_commit(v_empty(vs));
+              }
+            }
+            g += w.n_tiles;
+            for (int t = 0; t < w.nt; ++t) gt[t] += w.n_tiles;
+            continue;
           }
           for (int it = 0; it < w.n_tiles && ok; ++it) {
             const int64_t gi = g + it;
@@ -524,6 +580,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128 * t;
     const uint32_t tO = tmem + lane_off + C::kColO + DPAD * t;
+    const uint32_t tP = C::kSplitP ? tmem + lane_off + C::kColP + 64 * t : tS;  // where P goes
     const float sl2 = args.scale_log2;
     int64_t g = 0;  // key tiles of the units that include this query tile
     bool ok = true;
@@ -592,6 +649,12 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c]);
         }
+        if constexpr (C::kSplitP) {
+          // S has been read (the loads above waited for their data): the next
+          // S product may overwrite it
+          tc_fence_before();
+          mbar_arrive_warp(s_free(t));
+        }
         const bool full = tile_is_full(w.win, w.sq, w.sk, w.m0 + 128 * t, n0);
         if (!full) {
           const int32_t a = lo - n0, z = hi - n0;  // allowed columns [a, z]
@@ -625,6 +688,13 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
         // Scale-and-shift and the row sum run on packed fp32 pairs.
         uint64_t l4[4] = {0, 0, 0, 0};
         const uint64_t sl2x2 = f2_pack(sl2e, sl2e), negm2 = f2_pack(neg_m, neg_m);
+        if (C::kSplitP && it > 0) {
+          // P of the previous key tile must have been read by its P V product
+          // before this tile's P overwrites it
+          ok = mbar_wait(o_done(t), (uint32_t)((gi - 1) & 1), abort_flag, args.status, kSiteSoftmax);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           // Dropout: bit k of `keep` says whether column 32 c + k survives.
@@ -662,7 +732,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
             }
             packed[e] = pack2<BF16>(p0, p1);
           }
-          tmem_st16(tS + 16 * c, packed);
+          tmem_st16(tP + 16 * c, packed);
         }
         float la, lb, lc, ld;
         f2_unpack(f2_add(l4[0], l4[1]), la, lb);
