@@ -688,13 +688,6 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
         // Scale-and-shift and the row sum run on packed fp32 pairs.
         uint64_t l4[4] = {0, 0, 0, 0};
         const uint64_t sl2x2 = f2_pack(sl2e, sl2e), negm2 = f2_pack(neg_m, neg_m);
-        if (C::kSplitP && it > 0) {
-          // P of the previous key tile must have been read by its P V product
-          // before this tile's P overwrites it
-          ok = mbar_wait(o_done(t), (uint32_t)((gi - 1) & 1), abort_flag, args.status, kSiteSoftmax);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          tc_fence_after();
-        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           // Dropout: bit k of `keep` says whether column 32 c + k survives.
@@ -732,8 +725,18 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
             }
             packed[e] = pack2<BF16>(p0, p1);
           }
+          if (C::kSplitP && c == 0 && it > 0) {
+            // P of the previous key tile must have been read by its P V
+            // product before this tile's P overwrites it (waited for only now,
+            // after the first 32 columns' exponentials)
+            ok = mbar_wait(o_done(t), (uint32_t)((gi - 1) & 1), abort_flag, args.status,
+                           kSiteSoftmax);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+          }
           tmem_st16(tP + 16 * c, packed);
         }
+        if (!ok) break;
         float la, lb, lc, ld;
         f2_unpack(f2_add(l4[0], l4[1]), la, lb);
         f2_unpack(f2_add(l4[2], l4[3]), lc, ld);
