@@ -472,10 +472,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
                 if (t == w.nt - 1) tc_commit(v_empty(vs));
               }
             }
-            g += w.n_tiles;
-            for (int t = 0; t < w.nt; ++t) gt[t] += w.n_tiles;
-            continue;
-          }
+          } else {
           for (int it = 0; it < w.n_tiles && ok; ++it) {
             const int64_t gi = g + it;
             const int ks = (int)(gi % C::kKStages);
@@ -522,6 +519,7 @@ __global__ void __launch_bounds__(FwdCfg<NQ, DPAD, BIAS, DROPOUT>::kThreads, 1)
               issue_pv(t, vs, w.n_tiles > 1);
               if (t == w.nt - 1) tc_commit(v_empty(vs));
             }
+          }
           }
           g += w.n_tiles;
           for (int t = 0; t < w.nt; ++t) gt[t] += w.n_tiles;
