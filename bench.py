@@ -469,13 +469,40 @@ def peak_source(src, lowered, clocks):
 KERNEL_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu", "bwd.cu")
 
 
+def _code_only(text: str) -> str:
+    """C / C++ source without comments and with runs of whitespace collapsed:
+    what the compiler sees, so an edit of a comment keeps the hash."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":  # string or character literal, copied whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernels_sha256():
-    """Hash of the kernel sources, to tie committed counters to a kernel build."""
+    """Hash of the kernel sources (comments and layout ignored), to tie
+    committed counters to a kernel build."""
     import hashlib
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "scaled_dot_product_12_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "scaled_dot_product_12_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -2,29 +2,36 @@
 // FlashAttention after Tri Dao): tiled online softmax, O and LSE out.
 //
 // A persistent kernel: one CTA per SM walks a list of work units.  A unit is
-// NQ query tiles of 128 rows of one (sequence, head); its key tiles of 128 are
-// those the Generalized Sliding Window lets any of its rows see (mask.cuh),
-// and tiles with no masked pair skip the element test.  Units are numbered
-// query block fastest, so the CTAs running at one time share a few heads' K
-// and V in L2, and within a (sequence, head) longest first (the last query
-// block first, which under causal and bottom-right windows carries the most
-// key tiles); they are dealt to the CTAs round robin.  TMEM, the barriers
-// and the K / V rings live for the whole kernel; every barrier phase follows
-// one running count of key tiles, so the load of the next unit's tiles and
-// its first S product overlap the current unit's last softmax and epilogue.
+// NQ query tiles of 128 rows of one (sequence, head) (fewer where the
+// sequence ends); its key tiles of 128 are those the Generalized Sliding
+// Window lets any of its rows see (mask.cuh), and tiles with no masked pair
+// skip the element test.  Without a mask units are numbered query block
+// fastest, so the CTAs running at one time share a few heads' K and V in L2;
+// under a window query block slowest, most expensive first (longest
+// processing time first); they are dealt to the CTAs round robin, and a last
+// round at most half full is split into single-tile units.  TMEM, the
+// barriers and the K / V rings live for the whole kernel; every barrier
+// phase follows one running count of key tiles, so the load of the next
+// unit's tiles and its first S product overlap the current unit's last
+// softmax and epilogue.
 // Warp roles:
 //   warps 0..4*NQ-1  softmax: one 4-warp group per query tile, one row per
 //                    thread (TMEM lane = row); online exp2 softmax with lazy
-//                    rescaling, P written back into TMEM as 16-bit, O rescale
-//                    and the epilogue (and the zero rows of fully masked units);
+//                    rescaling (an additive bias added from shared memory),
+//                    P written into TMEM as 16-bit, O rescale and the
+//                    epilogue (and the zero rows of fully masked units);
 //   warp 4*NQ        TMA producer: Q once per unit (double-buffered at head
 //                    dims up to 64), K and V through separate rings;
 //   warp 4*NQ+1      MMA issuer (one thread): S = Q K^T (smem x smem) and
 //                    O += P V (P from TMEM, V from smem), TMEM owner;
-//   warps 4*NQ+2..   idle: they complete the producer / MMA warpgroup, whose
+//   warp 4*NQ+2      with a bias: TMA producer of the bias tiles;
+//   the rest         idle: they complete the producer / MMA warpgroup, whose
 //                    registers go to the softmax groups through setmaxnreg.
-// TMEM columns: S/P of tile t at [128 t, 128 t + 128), O of tile t at
-// [128 NQ + DPAD t, ...).
+// TMEM columns: S of tile t at [128 t, 128 t + 128); at head dim 128 P is
+// written over S and O of tile t sits at [128 NQ + 128 t, ...); at head dims
+// up to 64 P has columns of its own, [128 NQ + 64 t, ...), and O of tile t
+// follows at [192 NQ + 64 t, ...), so the next S product can be issued as
+// soon as the softmax has read S.
 #include <cuda_runtime.h>
 
 #include <type_traits>
