@@ -160,3 +160,14 @@ def test_end_to_end_groups_cover_the_workload_once():
         covered = [i for g in groups for i in range(size)[g]]
         assert covered == list(range(size)), name
         assert 1 <= len(groups) <= 4
+
+
+def test_kernel_hash_ignores_comments_but_not_code():
+    import bench
+    base = 'int f(int a) { return a + 1; }  // one\n/* two */ const char* s = "// x";\n'
+    same = '// header\nint f(int a)   {\n  return a + 1;  /* changed */ }\nconst char* s = "// x";'
+    other = 'int f(int a) { return a + 2; }  // one\n/* two */ const char* s = "// x";\n'
+    lit = 'int f(int a) { return a + 1; }  // one\n/* two */ const char* s = "// y";\n'
+    assert bench._code_only(base) == bench._code_only(same)
+    assert bench._code_only(base) != bench._code_only(other)
+    assert bench._code_only(base) != bench._code_only(lit)  # string contents are code
