@@ -466,7 +466,7 @@ def peak_source(src, lowered, clocks):
             f"{', '.join(seen) if seen else 'none'})")
 
 
-KERNEL_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu", "bwd.cu")
+KERNEL_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu", "fwd_pair.cu", "bwd.cu")
 
 
 def _code_only(text: str) -> str:

@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "fwd.cu", "fwd_pair.cu", "bwd.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "mask.cuh", "fwd.h"]
 LIB_NAME = "libattn.so"
 

@@ -191,7 +191,7 @@ bool bias_strides_ok(const int64_t* st, int64_t nb, int64_t nh, int64_t nrows, b
 }
 
 cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, int H, int B,
-                     const int64_t* st, bool packed) {
+                     const int64_t* st, bool packed, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const int64_t rows_c = rows > 0 ? rows : 1;
@@ -205,7 +205,7 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
   };
   cuuint64_t strides[3] = {pick(st[2], dims[1]), pick(st[1], dims[2]),
                            packed ? (cuuint64_t)16 : pick(st[0], dims[3])};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -331,6 +331,8 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
     cudaError_t e = make_map(&a.tq, p->q, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
     if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
     if (e == cudaSuccess) e = make_map(&a.tv, vbase, Dv, nk, p->H, p->B, p->v_stride, m.k_packed);
+    // half key tiles (64 rows) for the CTA-pair kernel
+    if (e == cudaSuccess) e = make_map(&a.tk2, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed, 64);
     if (e != cudaSuccess) return e;
     a.o = p->o;
     a.lse = p->lse;

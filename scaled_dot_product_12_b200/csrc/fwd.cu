@@ -820,6 +820,7 @@ static cudaError_t launch(const FwdArgs& args, int64_t n_units, cudaStream_t str
 }
 
 cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream) {
+  if (fwd_pair_eligible(args)) return launch_fwd_pair(args, stream);
   constexpr int NQ = 2;
   const int rows = 128 * NQ;
   const int64_t n_units = (int64_t)((args.Sq + rows - 1) / rows) * args.H * args.B;

@@ -14,6 +14,7 @@ namespace attn {
 // Boxes are 64 columns x 128 rows with 128-byte swizzle.
 struct FwdArgs {
   CUtensorMap tq, tk, tv;
+  CUtensorMap tk2;  // K with 64 x 64 boxes (the CTA-pair kernel loads half key tiles)
   void* o;
   float* lse;
   int64_t o_stride[3];
@@ -97,6 +98,9 @@ struct BwdArgs {
 };
 
 cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream);
+// The CTA-pair forward (dense, no mask, bias or dropout, head dims 128).
+bool fwd_pair_eligible(const FwdArgs& args);
+cudaError_t launch_fwd_pair(const FwdArgs& args, cudaStream_t stream);
 
 // Checks a kernel's register count at launch (the setmaxnreg splits assume
 // `min_regs` per thread; with fewer, the warpgroups that raise their count
