@@ -130,15 +130,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
   const bool leader = rank == 0;
   const int64_t pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int32_t n_mblocks = (args.Sq + 511) / 512;
-  const int64_t n_units = (int64_t)n_mblocks * args.H * args.B;
+  // Units: n_full of 512 rows (two query tiles per CTA), dealt round robin.
+  // When the last round would be at most half full, its units are split in
+  // two halves of 256 rows (one query tile per CTA), so that round takes
+  // about the time of one query tile's chain instead of two tiles'.
+  const int64_t n_full = (int64_t)n_mblocks * args.H * args.B;
+  const int64_t rounds = n_full / n_pairs, left = n_full - rounds * n_pairs;
+  const bool split = rounds >= 1 && left > 0 && 2 * left <= n_pairs;
+  const int64_t split_from = split ? rounds * n_pairs : n_full;
+  const int64_t n_units = split ? split_from + 2 * left : n_full;
   const int32_t n_tiles = (args.Sk + 127) / 128;
   if (sbase & 1023) {  // identical in both CTAs of the pair, so both return
     if (threadIdx.x == 0) atomicOr(args.status, 1u << kSiteTeardown);
     return;
   }
-  auto unit_of = [&](int64_t u, int32_t& b, int32_t& h, int32_t& m0) {
-    const int64_t hb = u / n_mblocks;
-    m0 = (int32_t)(u - hb * n_mblocks) * 512 + 256 * (int32_t)rank;  // this CTA's 256 rows
+  // Unit u: (batch b, head h), this CTA's first row m0 and its nt query
+  // tiles (rows m0 + 128 t); every role decodes the same units.
+  auto unit_of = [&](int64_t u, int32_t& b, int32_t& h, int32_t& m0, int& nt) {
+    int64_t fu = u;
+    int32_t half = 0;
+    nt = 2;
+    if (u >= split_from) {
+      fu = split_from + (u - split_from) / 2;
+      half = (int32_t)((u - split_from) & 1);
+      nt = 1;
+    }
+    const int64_t hb = fu / n_mblocks;
+    m0 = (int32_t)(fu - hb * n_mblocks) * 512 +
+         (nt == 2 ? 256 * (int32_t)rank : 256 * half + 128 * (int32_t)rank);
     h = (int32_t)(hb % args.H);
     b = (int32_t)(hb / args.H);
   };
@@ -209,17 +228,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
       prefetch_tmap(&args.tk2);
       prefetch_tmap(&args.tv);
       int64_t nk = 0, nv = 0, uc = 0;
+      int64_t qn0 = 0, qn1 = 0;  // Q loads issued per tile
       bool stop = false;
       for (int64_t u = pair; u < n_units && !stop; u += n_pairs) {
         int32_t b, h, m0;
-        unit_of(u, b, h, m0);
+        int nt;
+        unit_of(u, b, h, m0, nt);
         if (uc > 0 && !mbar_wait(q_empty, (uint32_t)((uc - 1) & 1), abort_flag, args.status, kSiteLoad))
           break;
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < nt; ++t) {
           if (leader) mbar_expect_tx(q_full(t), 2 * C::kQTile);
           for (int blk = 0; blk < 2; ++blk)
             tma_load_4d_pair(sQ + t * C::kQTile + blk * 16384, &args.tq, q_full(t), 64 * blk,
                              m0 + 128 * t, h, b);
+          ++(t == 0 ? qn0 : qn1);
         }
         ++uc;
         for (int it = 0; it < n_tiles; ++it) {
@@ -254,8 +276,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
           mbar_drain(k_full((int)(i % C::kStages)), (uint32_t)((i / C::kStages) & 1), args.status);
         for (int64_t i = nv > C::kStages ? nv - C::kStages : 0; i < nv; ++i)
           mbar_drain(v_full((int)(i % C::kStages)), (uint32_t)((i / C::kStages) & 1), args.status);
-        if (uc > 0)
-          for (int t = 0; t < 2; ++t) mbar_drain(q_full(t), (uint32_t)((uc - 1) & 1), args.status);
+        if (qn0 > 0) mbar_drain(q_full(0), (uint32_t)((qn0 - 1) & 1), args.status);
+        if (qn1 > 0) mbar_drain(q_full(1), (uint32_t)((qn1 - 1) & 1), args.status);
       }
     } else if (warp == 9 && lane == 0 && leader) {
       // ===================== MMA issuer (the leader) =====================
@@ -283,12 +305,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
                       idesc_o, (accumulate || kk > 0) ? 1u : 0u);
         commit_pair(o_done(t));
       };
-      int64_t g = 0, uc = 0;
-      bool ok = true;
-      for (int64_t u = pair; u < n_units && ok; u += n_pairs) {
-        for (int t = 0; t < 2 && ok; ++t)
-          ok = mbar_wait(q_full(t), (uint32_t)(uc & 1), abort_flag, args.status, kSiteMma);
-        ++uc;
+      // Phases: K / V rings follow the key tiles of all units (g); the S,
+      // P and O barriers of query tile t the key tiles of the units that
+      // include tile t (gt0, gt1); the Q barrier of tile t its loads (qn0,
+      // qn1).  The unit body is instantiated for two tiles and for one (a
+      // half unit), so its tile loops unroll and the counters stay in
+      // registers.
+      int64_t g = 0, gt0 = 0, gt1 = 0, qn0 = 0, qn1 = 0;
+      auto run_unit = [&](auto tiles) -> bool {
+        constexpr int NT = decltype(tiles)::value;
+        bool ok = true;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          int64_t& qn = t == 0 ? qn0 : qn1;
+          if (ok) ok = mbar_wait(q_full(t), (uint32_t)(qn & 1), abort_flag, args.status, kSiteMma);
+          ++qn;
+        }
         for (int it = 0; it < n_tiles && ok; ++it) {
           const int64_t gi = g + it;
           const int ks = (int)(gi % C::kStages);
@@ -296,17 +328,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
                                args.status, kSiteMma)))
             break;
           const int vs = (int)((gi - 1) % C::kStages);
-          for (int t = 0; t < 2 && ok; ++t) {
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            if (!ok) break;
             if (it > 0) {
-              if (!(ok = mbar_wait(p_ready(t), (uint32_t)((gi - 1) & 1), abort_flag,
-                                           args.status, kSiteMma)))
+              const int64_t gt = t == 0 ? gt0 : gt1;
+              if (!(ok = mbar_wait(p_ready(t), (uint32_t)((gt + it - 1) & 1), abort_flag,
+                                   args.status, kSiteMma)))
                 break;
               if (t == 0 && !(ok = mbar_wait(v_full(vs), (uint32_t)(((gi - 1) / C::kStages) & 1),
                                              abort_flag, args.status, kSiteMma)))
                 break;
               tc_fence_after();
               issue_pv(t, vs, it > 1);
-              if (t == 1) commit_pair(v_empty(vs));
+              if (t == NT - 1) commit_pair(v_empty(vs));
             }
             tc_fence_after();
             issue_s(t, ks);
@@ -318,19 +353,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
         if (ok) {
           const int64_t gl = g + n_tiles - 1;
           const int vs = (int)(gl % C::kStages);
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (!(ok = mbar_wait(p_ready(t), (uint32_t)(gl & 1), abort_flag, args.status,
-                                         kSiteMma)))
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            if (!ok) break;
+            const int64_t gt = t == 0 ? gt0 : gt1;
+            if (!(ok = mbar_wait(p_ready(t), (uint32_t)((gt + n_tiles - 1) & 1), abort_flag,
+                                 args.status, kSiteMma)))
               break;
             if (t == 0 && !(ok = mbar_wait(v_full(vs), (uint32_t)((gl / C::kStages) & 1), abort_flag,
                                            args.status, kSiteMma)))
               break;
             tc_fence_after();
             issue_pv(t, vs, n_tiles > 1);
-            if (t == 1) commit_pair(v_empty(vs));
+            if (t == NT - 1) commit_pair(v_empty(vs));
           }
         }
         g += n_tiles;
+        gt0 += n_tiles;
+        if (NT == 2) gt1 += n_tiles;
+        return ok;
+      };
+      bool ok = true;
+      for (int64_t u = pair; u < n_units && ok; u += n_pairs) {
+        int32_t b, h, m0;
+        int nt;
+        unit_of(u, b, h, m0, nt);
+        ok = nt == 2 ? run_unit(std::integral_constant<int, 2>{})
+                     : run_unit(std::integral_constant<int, 1>{});
       }
       // every product issued has completed before TMEM is released
       commit_pair(mma_done);
@@ -346,11 +395,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
     const uint32_t tS = tmem + lane_off + 128 * t;
     const uint32_t tO = tmem + lane_off + C::kColO + 128 * t;
     const float sl2 = args.scale_log2;
-    int64_t g = 0;
+    int64_t g = 0;  // key tiles of the units that include this query tile
     bool ok = true;
     for (int64_t u = pair; u < n_units && ok; u += n_pairs) {
       int32_t b, h, m0;
-      unit_of(u, b, h, m0);
+      int nt;
+      unit_of(u, b, h, m0, nt);
+      if (t >= nt) continue;  // a half unit: tile 0 only
       const int32_t i = m0 + 128 * t + r;
       const bool valid = i < args.Sq;
       float m_used = -INFINITY, l = 0.f;

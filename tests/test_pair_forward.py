@@ -2,6 +2,7 @@
 dropout, head dims 128: the calls the library routes to the two-SM kernel)
 against the fp64 oracle, on shapes that stress what that kernel adds: many
 512-row units per CTA pair (persistent loop, Q buffers reused across units),
+a last round split into 256-row half units,
 units whose second CTA has no valid rows, ragged key tiles, a single query
 row, fp16 with a negative scale and the TH LSE layout, and strided views."""
 
@@ -19,6 +20,7 @@ CASES = [
     (1, 3, 1, 5000, torch.bfloat16, None, "HT"),       # one query row
     (2, 2, 4096, 129, torch.bfloat16, 0.3, "HT"),      # second key tile holds one key
     (1, 1, 512, 512, torch.float16, None, "HT"),       # exactly one unit
+    (1, 80, 1000, 300, torch.bfloat16, None, "HT"),    # 160 units: last round in half units
 ]
 
 
