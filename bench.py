@@ -218,6 +218,14 @@ def workload_bytes(w: synth.Workload):
             "bwd_other": rq * (14 * D + 4)}
 
 
+def fwd_kernel_name(w: synth.Workload, bias: bool) -> str:
+    """The forward kernel the library runs for this workload: the CTA-pair
+    kernel for dense calls at head dim 128 with no window, bias or dropout,
+    the one-CTA kernel otherwise (the dispatch rule of the forward launch)."""
+    dense = not w.packed and w.window_left == synth.WINDOW_INF and w.window_right == synth.WINDOW_INF
+    return "attn_fwd_pair_kernel" if dense and w.D == 128 and not bias else "attn_fwd_kernel"
+
+
 def describe(w: synth.Workload):
     sq, sk = seqlens(w)
     layout = ("packed 1THD with cumulative seqlens, LSE TH" if w.packed
@@ -391,8 +399,8 @@ def run_gpu(args, rank, world, local):
         roof = kernel_roofline("attn_bwd_kernel", bwd_flops, nbytes["attn_bwd_kernel"], main_ms,
                                peak, hbm)
     else:
-        roof = kernel_roofline("attn_fwd_kernel", fwd_flops, nbytes["attn_fwd_kernel"], fwd_ms,
-                               peak, hbm)
+        roof = kernel_roofline(fwd_kernel_name(w, args.bias), fwd_flops, nbytes["attn_fwd_kernel"],
+                               fwd_ms, peak, hbm)
     roof["peak_source"] = peak_source(peak_src, lowered, clock_summary)
     roof["traffic"] = load_traffic(roof["kernel"], w.name)
 
@@ -466,7 +474,17 @@ def peak_source(src, lowered, clocks):
             f"{', '.join(seen) if seen else 'none'})")
 
 
-KERNEL_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu", "fwd_pair.cu", "bwd.cu")
+# The sources each kernel is compiled from (its .cu file and the headers it
+# includes): committed counters of a kernel stay valid while these are unchanged.
+_BWD_SOURCES = ("common.cuh", "mask.cuh", "fwd.h", "bwd.cu")
+KERNEL_SOURCES_BY_KERNEL = {
+    "attn_fwd_kernel": ("common.cuh", "mask.cuh", "fwd.h", "fwd.cu"),
+    "attn_fwd_pair_kernel": ("common.cuh", "fwd.h", "fwd_pair.cu"),
+    "attn_bwd_kernel": _BWD_SOURCES,
+    "attn_bwd_pre_kernel": _BWD_SOURCES,
+    "attn_dq_convert_kernel": _BWD_SOURCES,
+}
+KERNEL_SOURCES = tuple(sorted({f for v in KERNEL_SOURCES_BY_KERNEL.values() for f in v}))
 
 
 def _code_only(text: str) -> str:
@@ -495,12 +513,12 @@ def _code_only(text: str) -> str:
     return re.sub(r"\s+", " ", "".join(out)).strip()
 
 
-def kernels_sha256():
-    """Hash of the kernel sources (comments and layout ignored), to tie
-    committed counters to a kernel build."""
+def kernels_sha256(kernel=None):
+    """Hash of a kernel's sources (comments and layout ignored; all kernel
+    sources when `kernel` is None), to tie committed counters to a build."""
     import hashlib
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES_BY_KERNEL[kernel] if kernel else KERNEL_SOURCES:
         with open(os.path.join(ROOT, "scaled_dot_product_12_b200", "csrc", name)) as f:
             h.update(_code_only(f.read()).encode())
     return h.hexdigest()
@@ -515,7 +533,9 @@ def load_traffic(kernel, workload):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("kernels_sha256") != kernels_sha256():
+    if kernel not in KERNEL_SOURCES_BY_KERNEL:
+        return None
+    if d.get("kernels_sha256", {}).get(kernel) != kernels_sha256(kernel):
         return None
     return d.get("bytes_per_launch", {}).get(f"{kernel}:{workload}")
 

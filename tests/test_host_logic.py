@@ -139,14 +139,29 @@ def test_traffic_is_null_for_other_kernel_builds(tmp_path, monkeypatch):
     for name in bench.KERNEL_SOURCES:
         (src / name).write_text(name)
     monkeypatch.setattr(bench, "ROOT", str(root))
-    good = bench.kernels_sha256()
-    table = {"attn_bwd_kernel:ltx_15300": 123}
+    hashes = {k: bench.kernels_sha256(k) for k in ("attn_bwd_kernel", "attn_fwd_pair_kernel")}
+    table = {"attn_bwd_kernel:ltx_15300": 123, "attn_fwd_pair_kernel:ltx_15300": 45}
     (root / "profiles" / "traffic.json").write_text(
-        json.dumps({"kernels_sha256": good, "bytes_per_launch": table}))
+        json.dumps({"kernels_sha256": hashes, "bytes_per_launch": table}))
     assert bench.load_traffic("attn_bwd_kernel", "ltx_15300") == 123
-    assert bench.load_traffic("attn_fwd_kernel", "ltx_15300") is None
-    (src / "bwd.cu").write_text("changed")
+    assert bench.load_traffic("attn_fwd_pair_kernel", "ltx_15300") == 45
+    assert bench.load_traffic("attn_fwd_kernel", "ltx_15300") is None  # no record
+    # a change to one kernel's source voids its counters, not another's
+    (src / "fwd_pair.cu").write_text("changed")
+    assert bench.load_traffic("attn_fwd_pair_kernel", "ltx_15300") is None
+    assert bench.load_traffic("attn_bwd_kernel", "ltx_15300") == 123
+    (src / "common.cuh").write_text("changed")
     assert bench.load_traffic("attn_bwd_kernel", "ltx_15300") is None
+
+
+def test_forward_kernel_name_follows_the_dispatch_rule():
+    """Dense calls at D = 128 without a window or bias run the CTA-pair kernel."""
+    w = synth.ALL_WORKLOADS
+    assert bench.fwd_kernel_name(w["ltx_15300"], False) == "attn_fwd_pair_kernel"
+    assert bench.fwd_kernel_name(w["ltx_15300"], True) == "attn_fwd_kernel"
+    assert bench.fwd_kernel_name(w["bert_large"], False) == "attn_fwd_kernel"
+    assert bench.fwd_kernel_name(w["gpt2"], False) == "attn_fwd_kernel"
+    assert bench.fwd_kernel_name(w["varlen_D128_w256_0_TL"], False) == "attn_fwd_kernel"
 
 
 def test_end_to_end_groups_cover_the_workload_once():
