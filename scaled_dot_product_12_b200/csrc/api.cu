@@ -328,12 +328,6 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
     const void* kbase = rows_k > 0 ? p->k : p->q;
     const void* vbase = rows_k > 0 ? p->v : p->q;
     const int Dv = p->Dv ? p->Dv : p->D;
-    cudaError_t e = make_map(&a.tq, p->q, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
-    if (e == cudaSuccess) e = make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
-    if (e == cudaSuccess) e = make_map(&a.tv, vbase, Dv, nk, p->H, p->B, p->v_stride, m.k_packed);
-    // half key tiles (64 rows) for the CTA-pair kernel
-    if (e == cudaSuccess) e = make_map(&a.tk2, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed, 64);
-    if (e != cudaSuccess) return e;
     a.o = p->o;
     a.lse = p->lse;
     for (int i = 0; i < 3; ++i) a.o_stride[i] = p->o_stride[i];
@@ -374,11 +368,18 @@ int attn_fwd(const attn_fwd_params* params, void* stream_ptr) {
     set_dropout(a, p);
     a.bias = p->bias;
     for (int i = 0; i < 3; ++i) a.bias_stride[i] = p->bias_stride[i];
-    if (p->bias) {
+    // K is read in 128-row tiles by the one-CTA kernel and in 64-row halves
+    // by the CTA-pair kernel: only the map of the kernel that runs is encoded.
+    const bool pair = attn::fwd_pair_eligible(a);
+    cudaError_t e = make_map(&a.tq, p->q, p->D, nq, p->H, p->B, p->q_stride, m.q_packed);
+    if (e == cudaSuccess)
+      e = pair ? make_map(&a.tk2, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed, 64)
+               : make_map(&a.tk, kbase, p->D, nk, p->H, p->B, p->k_stride, m.k_packed);
+    if (e == cudaSuccess) e = make_map(&a.tv, vbase, Dv, nk, p->H, p->B, p->v_stride, m.k_packed);
+    if (e == cudaSuccess && p->bias)
       e = make_bias_map(&a.tb, p->bias, p->Sq, p->Sk, p->H, p->B, p->bias_stride, &a.bias_h_bcast,
                         &a.bias_b_bcast);
-      if (e != cudaSuccess) return e;
-    }
+    if (e != cudaSuccess) return e;
     return attn::launch_fwd(a, stream);
   });
 }

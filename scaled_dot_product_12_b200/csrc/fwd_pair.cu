@@ -530,6 +530,7 @@ static cudaError_t launch_pair(const FwdArgs& args, cudaStream_t stream) {
   // cluster group), asked once per device: more would run as a second wave.
   static std::atomic<int> resident[64];
   const int64_t n_units = (int64_t)((args.Sq + 511) / 512) * args.H * args.B;
+  if (n_units <= 0) return cudaSuccess;
   return prepared_launch(kern, prepared, args.dev, C::kSmemBytes, C::kLaunchRegs, [&] {
     const bool cache = args.dev >= 0 && args.dev < 64;
     int pairs = cache ? resident[args.dev].load(std::memory_order_relaxed) : 0;

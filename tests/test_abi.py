@@ -108,6 +108,15 @@ def test_forward_rejects_invalid_parameters(B, field, value):
     assert _call_fwd(B, _fwd(B, **{field: value})) == B.ERROR_INVALID_VALUE
 
 
+def test_empty_head_dim_128_problems_succeed_without_a_device(B):
+    # dense D = 128 calls go to the CTA-pair kernel: an empty batch or head
+    # count returns before any launch, as for every other kernel
+    st = (3 * 128 * 128, 128 * 128, 128)
+    for kw in ({"B": 0}, {"H": 0}, {"B": 0, "H": 0}):
+        p = _fwd(B, D=128, q_stride=st, k_stride=st, v_stride=st, o_stride=st, **kw)
+        assert _call_fwd(B, p) == 0
+
+
 def test_version_one_callers_are_accepted(B):
     # a caller built against version 1 passes version 1 and the version-1 size:
     # the call validates (an empty problem succeeds without a device) ...
