@@ -1,7 +1,7 @@
 // FlashAttention forward on CTA pairs: the same online softmax and the same
 // warp roles as fwd.cu, with every product issued once for two SMs (tcgen05
 // with cta_group::2, M = 256).  Used for dense inputs without a mask, bias or
-// dropout at head dims 128, the case whose time is spent in the products and
+// dropout at head dim 128, the case whose time is spent in the products and
 // the exponentials.
 //
 // A pair works on 512 query rows of one (batch, head): CTA r holds query
@@ -20,8 +20,9 @@
 // products is signalled to both CTAs (multicast commit); both CTAs' loads
 // complete on the leader's barriers, whose transaction counts the leader
 // sets for both; the softmax warps of both CTAs report P ready to the
-// leader's barriers.  Units (512 rows) are dealt to the pairs round robin;
-// every barrier's phase follows a running count of key tiles over them.
+// leader's barriers.  Units (512 rows; a last round at most half full in
+// 256-row halves, one query tile per CTA) are dealt to the pairs round
+// robin; every barrier's phase follows a running count of key tiles.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
