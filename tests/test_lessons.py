@@ -191,13 +191,14 @@ def test_window_zero_zero_keeps_fp16_subnormals(packed, br):
                 assert (row == 0).all()
 
 
-def test_null_logsumexp_pointer():
+@pytest.mark.parametrize("wl,wr,br", [(256, 0, True), (INF, INF, False)])  # the latter: CTA pairs
+def test_null_logsumexp_pointer(wl, wr, br):
     B = binding()
     dev = torch.device("cuda")
     q, k, v, _ = dense_inputs(2, 2, 300, 400, 128, torch.bfloat16, 61)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    o1, lse = B.forward(qd, kd, vd, sm_scale=0.09, window=(256, 0), bottom_right=True)
-    o2, none = B.forward(qd, kd, vd, sm_scale=0.09, window=(256, 0), bottom_right=True,
+    o1, lse = B.forward(qd, kd, vd, sm_scale=0.09, window=(wl, wr), bottom_right=br)
+    o2, none = B.forward(qd, kd, vd, sm_scale=0.09, window=(wl, wr), bottom_right=br,
                          return_lse=False)
     torch.cuda.synchronize()
     assert none is None and torch.equal(o1, o2)
