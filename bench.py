@@ -220,10 +220,12 @@ def workload_bytes(w: synth.Workload):
 
 def fwd_kernel_name(w: synth.Workload, bias: bool) -> str:
     """The forward kernel the library runs for this workload: the CTA-pair
-    kernel for dense calls at head dim 128 with no window, bias or dropout,
-    the one-CTA kernel otherwise (the dispatch rule of the forward launch)."""
+    kernel for dense calls with head dims above 64 (the value head dim a
+    multiple of 16) and no window, bias or dropout, the one-CTA kernel
+    otherwise (the dispatch rule of the forward launch)."""
     dense = not w.packed and w.window_left == synth.WINDOW_INF and w.window_right == synth.WINDOW_INF
-    return "attn_fwd_pair_kernel" if dense and w.D == 128 and not bias else "attn_fwd_kernel"
+    pair = dense and 64 < w.D <= 128 and w.D % 16 == 0 and not bias
+    return "attn_fwd_pair_kernel" if pair else "attn_fwd_kernel"
 
 
 def describe(w: synth.Workload):

@@ -98,7 +98,8 @@ struct BwdArgs {
 };
 
 cudaError_t launch_fwd(const FwdArgs& args, cudaStream_t stream);
-// The CTA-pair forward (dense, no mask, bias or dropout, head dims 128).
+// The CTA-pair forward (dense, no mask, bias or dropout, the wider head dim
+// in (64, 128], Dv a multiple of 16).
 bool fwd_pair_eligible(const FwdArgs& args);
 cudaError_t launch_fwd_pair(const FwdArgs& args, cudaStream_t stream);
 

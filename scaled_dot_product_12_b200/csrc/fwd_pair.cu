@@ -1,8 +1,8 @@
 // FlashAttention forward on CTA pairs: the same online softmax and the same
 // warp roles as fwd.cu, with every product issued once for two SMs (tcgen05
 // with cta_group::2, M = 256).  Used for dense inputs without a mask, bias or
-// dropout at head dim 128, the case whose time is spent in the products and
-// the exponentials.
+// dropout whose head dims take 128-column tiles (the long head-dim-128
+// workloads, whose time is spent in the products and the exponentials).
 //
 // A pair works on 512 query rows of one (batch, head): CTA r holds query
 // tiles [256 r, 256 r + 256) of them as two 128-row tiles, like one CTA of
@@ -493,6 +493,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint8_t* orow = valid ? o_row_ptr(b, h, i) : nullptr;
+        // O / l to 16 bits, 16 columns at a time up to Dv (a multiple of 16;
+        // the columns past it are TMA fill and not stored)
         for (int c = 0; c < 8; ++c) {
           uint32_t rr[16];
           tmem_ld16(tO + 16 * c, rr);
@@ -500,7 +502,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             pk[e] = pack2<BF16>(__uint_as_float(rr[2 * e]) * inv, __uint_as_float(rr[2 * e + 1]) * inv);
-          if (valid) st_row16(orow, c, pk, 128);
+          if (valid && 16 * c < args.Dv) {
+            st_global_v4(orow + 32 * c, pk[0], pk[1], pk[2], pk[3]);
+            st_global_v4(orow + 32 * c + 16, pk[4], pk[5], pk[6], pk[7]);
+          }
         }
         if (valid && args.lse)
           *lse_ptr(b, h, i) = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -553,9 +558,15 @@ static cudaError_t launch_pair(const FwdArgs& args, cudaStream_t stream) {
   });
 }
 
+// Dense calls without a window, bias or dropout whose head dims take the
+// 128-column tiles (the wider of D and Dv above 64; TMA fills the columns past
+// a tensor's own head dim with zeros) and whose O rows end on a 16-column
+// boundary (Dv a multiple of 16: O is stored in whole 16-column chunks).
 bool fwd_pair_eligible(const FwdArgs& a) {
-  return a.D == 128 && a.Dv == 128 && !a.q_packed && !a.k_packed && !a.q_padded && !a.k_padded &&
-         a.wl == 2147483647 && a.wr == 2147483647 && !a.dropout && !a.bias && a.Sq > 0 && a.Sk > 0;
+  return (a.D > 64 || a.Dv > 64) && a.D <= 128 && a.Dv <= 128 && a.Dv % 16 == 0 &&
+         !a.q_packed && !a.k_packed &&
+         !a.q_padded && !a.k_padded && a.wl == 2147483647 && a.wr == 2147483647 && !a.dropout &&
+         !a.bias && a.Sq > 0 && a.Sk > 0;
 }
 
 cudaError_t launch_fwd_pair(const FwdArgs& args, cudaStream_t stream) {

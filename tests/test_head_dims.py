@@ -81,7 +81,11 @@ def test_packed_head_dims(D):
     assert_grads([f64(t) for t in (dq, dk, dv)], [want["dq"], want["dk"], want["dv"]])
 
 
-@pytest.mark.parametrize("D,Dv", [(64, 128), (128, 64), (48, 80), (67, 13), (128, 32), (16, 120)])
+# Without a window, the pairs whose value head dim is a multiple of 16 and whose
+# wider head dim is above 64 run on the CTA-pair forward: (64, 128), (128, 64),
+# (48, 80), (128, 32), (80, 80), (96, 96), (112, 112), (88, 96), (72, 128).
+@pytest.mark.parametrize("D,Dv", [(64, 128), (128, 64), (48, 80), (67, 13), (128, 32), (16, 120),
+                                  (80, 80), (96, 96), (112, 112), (88, 96), (72, 128)])
 @pytest.mark.parametrize("w", [(INF, INF, False), (CTL, 0, False), (256, 0, True)], ids=str)
 def test_value_head_dim_of_its_own(D, Dv, w):
     # Hdim_vo != Hdim_qk (AOTriton 0.15b release notes, "Kernel Bug Fixes"):
