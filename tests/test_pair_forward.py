@@ -1,6 +1,7 @@
 """GPU parity of the CTA-pair forward (dense inputs, no window, bias or
-dropout, head dims 128: the calls the library routes to the two-SM kernel)
-against the fp64 oracle, on shapes that stress what that kernel adds: many
+dropout, head dims above 64: the calls the library routes to the two-SM
+kernel; here D = 128, the other head dims are in test_head_dims.py) against
+the fp64 oracle, on shapes that stress what that kernel adds: many
 512-row units per CTA pair (persistent loop, Q buffers reused across units),
 a last round split into 256-row half units,
 units whose second CTA has no valid rows, ragged key tiles, a single query
